@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated DeltaNet core on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdn|reference]
+
+One step = one pass of the whole prefill path over one batch: the gates
+(gdn_gates) and the chunked prefill (gdn_chunk_prefill) over the long-context
+workload B=1, T=32768, 16 q/k heads, 32 value heads, d=128, bf16, BT=64
+(synthetic, seeded).  The JSON line's ``value`` is prefill tokens/s over all
+ranks.  The decode step (B=64, H=32, d=128, fp32 state, 1024 consecutive steps)
+is measured in the same run and reported under ``decode`` with its HBM roofline.
+
+Under torchrun every rank runs its own independent replica of the workload (the
+path needs no exchange between GPUs); the step time is the max over ranks.
+
+``--impl reference`` times the CPU fp64 oracle instead, on the host cores, on a
+bounded prefix of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s @32K,H32,d128; decode-step HBM GB/s vs peak"
+PREFILL = dict(B=1, T=32768, HK=16, HV=32, D=128, BT=64)
+DECODE = dict(B=64, H=32, D=128, steps=1024)
+WORKLOAD = "long prefill: B=1 T=32768 HK=16 HV=32 Dk=Dv=128 bf16 BT=64, fp32 state, zero initial state"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def prefill_flops_per_token(HK, HV, D, C):
+    """Contraction FLOPs of the chunked form per token (a formula, not a count of
+    what a kernel executes): per value head 6 C d (W, U, P Delta) + 6 d^2
+    (W H, Q H, K^T Delta) + C^2 / 3 (triangular solve); per q/k head 4 C d
+    (K K^T and Q K^T)."""
+    return HV * (6 * C * D + 6 * D * D + C * C / 3.0) + HK * (4 * C * D)
+
+
+def prefill_bytes_per_token(HK, HV, D, io_bytes=2):
+    """Algorithmic HBM bytes per token: read q, k, v, g, beta; write o."""
+    return 2 * HK * D * io_bytes + HV * D * io_bytes + 2 * HV * 4 + HV * D * io_bytes
+
+
+def decode_bytes_per_step(B, HK, HV, Dk, Dv, io_bytes=2):
+    """State read + write (fp32), q, k, v read, o written, g and beta read."""
+    return (2 * B * HV * Dk * Dv * 4 + 2 * B * HK * Dk * io_bytes + 2 * B * HV * Dv * io_bytes
+            + 2 * B * HV * 4)
+
+
+# ---------------------------------------------------------------------------
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        exe = shutil.which("nvidia-smi")
+        if not exe:
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        self.proc = subprocess.Popen([exe, f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                      "-i", str(self.dev), "-lms", "100"],
+                                     stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r["power"] > 0.5 * max(x["power"] for x in rows)] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": rows[0]["smax"],
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+def cpu_oracle_sample(target_s: float, T_max: int):
+    """Time the oracle (gates + recurrence, fp64, all host cores) on a prefix of
+    the long workload sized to about ``target_s`` seconds.  Returns
+    (tokens/s, tokens, seconds, threads)."""
+    import numpy as np
+    import oracle
+    from gated_deltanet_sequence_delta_b200 import inputs as I
+    probe_T = 64
+    inp = I.make_prefill(1, probe_T, PREFILL["HK"], PREFILL["HV"], PREFILL["D"], PREFILL["D"],
+                         io_dtype=I.BF16, seed=2)
+
+    def run(inp):
+        q, k, v = inp.q.f64(), inp.k.f64(), inp.v.f64()
+        t0 = time.perf_counter()
+        g, beta = oracle.gates(inp.a.astype(np.float64), inp.b.astype(np.float64),
+                               inp.A_log.astype(np.float64), inp.dt_bias.astype(np.float64))
+        oracle.recurrence(q, k, v, g, beta, scale=1.0, l2norm=True)
+        return time.perf_counter() - t0
+
+    run(inp)
+    t = run(inp)
+    T_s = int(min(T_max, max(probe_T, probe_T * target_s / max(t, 1e-6))))
+    T_s = max(64, (T_s // 64) * 64)
+    inp = I.make_prefill(1, T_s, PREFILL["HK"], PREFILL["HV"], PREFILL["D"], PREFILL["D"],
+                         io_dtype=I.BF16, seed=2)
+    t = run(inp)
+    return T_s / t, T_s, t, oracle.max_threads()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    # size each step so that warmup + steps stay within about two minutes
+    per_step = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(per_step, PREFILL["T"])
+    vals, toks, secs = [], [], []
+    threads = None
+    for _ in range(args.steps):
+        v, T_s, t, threads = cpu_oracle_sample(per_step, PREFILL["T"])
+        vals.append(v)
+        toks.append(T_s)
+        secs.append(t)
+    value = sum(toks) / sum(secs)
+    sample = (f"first {toks[0]} tokens of the T=32768 workload per step (all 32 value heads), "
+              f"gates + fp64 recurrence")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(secs) / len(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_step": toks[0], "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def run_gdn(args, rank, world, dist):
+    import numpy as np
+    import torch
+    import gated_deltanet_sequence_delta_b200 as G
+    from gated_deltanet_sequence_delta_b200 import binding
+    from gated_deltanet_sequence_delta_b200 import inputs as I
+
+    binding.lib()  # fails loudly if the CUDA library is not built
+    dev = torch.device("cuda", torch.cuda.current_device())
+    P, pk = peaks()
+
+    def dev_t(t):
+        if isinstance(t, I.Tensor):
+            if t.dtype == I.BF16:
+                return torch.from_numpy(t.data.view(np.int16)).view(torch.bfloat16).to(dev)
+            return torch.from_numpy(t.data).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(t)).to(dev)
+
+    def pinned(t):
+        if isinstance(t, I.Tensor):
+            if t.dtype == I.BF16:
+                return torch.from_numpy(t.data.view(np.int16)).view(torch.bfloat16).pin_memory()
+            return torch.from_numpy(t.data).pin_memory()
+        return torch.from_numpy(np.ascontiguousarray(t)).pin_memory()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    T, HK, HV, D, BT = PREFILL["T"], PREFILL["HK"], PREFILL["HV"], PREFILL["D"], PREFILL["BT"]
+    do_prefill = args.only in ("all", "prefill")
+    do_decode = args.only in ("all", "decode")
+    clocks = Clocks(torch.cuda.current_device())
+    line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic"}
+    if do_prefill:
+        clocks.start()
+        line.update(bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_over_ranks))
+    if do_decode:
+        if not do_prefill:
+            clocks.start()
+        line["decode"] = bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks)
+    line["clocks"] = clocks.stop()
+    if do_prefill and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, T_s, t, th = cpu_oracle_sample(args.cpu_seconds, T)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": th, "kind": "oracle",
+                                "sample": f"first {T_s} tokens of the workload, all 32 value heads, "
+                                          f"gates + fp64 recurrence, {t:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _traffic():
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        return json.load(open(prof))
+    return {}
+
+
+def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_over_ranks):
+    import numpy as np
+    import statistics
+    import torch
+    import gated_deltanet_sequence_delta_b200 as G
+    from gated_deltanet_sequence_delta_b200 import inputs as I
+    T, HK, HV, D, BT = PREFILL["T"], PREFILL["HK"], PREFILL["HV"], PREFILL["D"], PREFILL["BT"]
+    inp = I.make_prefill(1, T, HK, HV, D, D, io_dtype=I.BF16, seed=2 + 1000 * rank, BT=BT, name="long")
+    q, k, v = dev_t(inp.q), dev_t(inp.k), dev_t(inp.v)
+    a, b = dev_t(inp.a), dev_t(inp.b)
+    A_log, dt_bias = dev_t(inp.A_log), dev_t(inp.dt_bias)
+    g = torch.empty((1, T, HV), dtype=torch.float32, device=dev)
+    beta = torch.empty_like(g)
+    o = torch.empty((1, T, HV, D), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((1, HV, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(G.prefill_workspace_bytes(T, 1, HK, HV, D, D, BT, 1), dtype=torch.uint8, device=dev)
+
+    def prefill_step(evs=None):
+        G.gdn_gates(a, b, A_log, dt_bias, g=g, beta=beta)
+        if evs is not None:
+            evs[0].record()
+        G.gdn_chunk_prefill(q, k, v, g, beta, BT=BT, o=o, final_state=hT, workspace=ws)
+        if evs is not None:
+            evs[1].record()
+
+    for _ in range(max(3, args.warmup)):
+        prefill_step()
+    barrier()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    n0 = G.kernel_launches()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        prefill_step(kev[i])
+    t1.record()
+    barrier()
+    launches = G.kernel_launches() - n0
+    ms_local = t0.elapsed_time(t1) / args.steps
+    kernel_ms_local = statistics.mean(e0.elapsed_time(e1) for e0, e1 in kev)
+    ms = max_over_ranks(ms_local)
+    kernel_ms = max_over_ranks(kernel_ms_local)
+
+    # ---------------- e2e through host buffers ----------------
+    hq, hk_, hv = pinned(inp.q), pinned(inp.k), pinned(inp.v)
+    ha, hb = pinned(inp.a), pinned(inp.b)
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hh = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk_, hv, ha, hb))
+    d2h = ho.numel() * ho.element_size() + hh.numel() * hh.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        a.copy_(ha, non_blocking=True)
+        b.copy_(hb, non_blocking=True)
+        prefill_step()
+        ho.copy_(o, non_blocking=True)
+        hh.copy_(hT, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    del hq, hk_, hv, ha, hb, ho, hh
+    flops = prefill_flops_per_token(HK, HV, D, BT) * T
+    pbytes = prefill_bytes_per_token(HK, HV, D) * T + HV * D * D * 4
+    tflops = flops / (kernel_ms * 1e-3) / 1e12
+    peak_tf = P["bf16_tflops"]
+    return {
+        "value": world * T / (ms * 1e-3), "ms_per_step": ms,
+        "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": T,
+                   "l2": "no flush: each step reads/writes ~0.8 GB, over 6x the 126 MB L2",
+                   "parallelism": f"replicas x{world} (independent problems, no collective)"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": tflops / peak_tf, "traffic": _traffic().get("prefill_bytes_per_launch"),
+                     "peak_kind": f"{pk} bf16 dense (burst)",
+                     "flops_per_launch": flops, "kernel_ms": kernel_ms,
+                     "hbm_view": {"achieved_gbs": pbytes / (kernel_ms * 1e-3) / 1e9,
+                                  "peak_gbs": P["hbm_gbs"],
+                                  "frac": pbytes / (kernel_ms * 1e-3) / 1e9 / P["hbm_gbs"],
+                                  "bytes_per_launch": pbytes}},
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches,
+    }
+
+
+def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks):
+    import torch
+    import gated_deltanet_sequence_delta_b200 as G
+    from gated_deltanet_sequence_delta_b200 import inputs as I
+    ds = I.decode(B=DECODE["B"], H=DECODE["H"], D=DECODE["D"], seed=1 + 1000 * rank)
+    ring = []
+    for s in range(8):
+        dq, dk, dv, da, db = ds.step(s)
+        ring.append((dev_t(dq), dev_t(dk), dev_t(dv), dev_t(da), dev_t(db)))
+    state = dev_t(ds.state0)
+    dA, dbias = dev_t(ds.A_log), dev_t(ds.dt_bias)
+    dg = torch.empty((ds.B, ds.HV), dtype=torch.float32, device=dev)
+    dbeta = torch.empty_like(dg)
+    do = torch.empty((ds.B, ds.HV, ds.Dv), dtype=torch.bfloat16, device=dev)
+
+    def decode_step(i):
+        dq, dk, dv, da, db = ring[i % len(ring)]
+        G.gdn_gates(da, db, dA, dbias, g=dg, beta=dbeta)
+        G.gdn_decode_step(dq, dk, dv, dg, dbeta, state, o=do)
+
+    for i in range(5):
+        decode_step(i)
+    barrier()
+    n_dec = args.decode_steps
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    nd0 = G.kernel_launches()
+    d0.record()
+    for i in range(n_dec):
+        decode_step(i)
+    d1.record()
+    barrier()
+    dec_launches = G.kernel_launches() - nd0
+    dec_ms = max_over_ranks(d0.elapsed_time(d1) / n_dec)
+    # the decode kernel alone, same inputs, back to back
+    dq, dk, dv, _, _ = ring[0]
+    k0 = torch.cuda.Event(enable_timing=True)
+    k1 = torch.cuda.Event(enable_timing=True)
+    k0.record()
+    for i in range(n_dec):
+        G.gdn_decode_step(dq, dk, dv, dg, dbeta, state, o=do)
+    k1.record()
+    barrier()
+    dec_kernel_ms = max_over_ranks(k0.elapsed_time(k1) / n_dec)
+    dbytes = decode_bytes_per_step(ds.B, ds.HK, ds.HV, ds.Dk, ds.Dv)
+    dgbs = dbytes / (dec_kernel_ms * 1e-3) / 1e9
+    return {"workload": "decode: B=64 HK=HV=32 Dk=Dv=128 bf16 q/k/v, fp32 state 128 MiB, "
+                        f"{n_dec} consecutive steps (gates + step), inputs cycled from 8 resident steps",
+            "ms_per_step": dec_ms, "steps_per_s": world * 1e3 / dec_ms,
+            "tokens_per_s": world * ds.B * 1e3 / dec_ms,
+            "gpu_launches": dec_launches,
+            "roofline": {"bound": "hbm", "achieved": dgbs, "peak": P["hbm_gbs"], "unit": "GB/s",
+                         "frac": dgbs / P["hbm_gbs"],
+                         "traffic": _traffic().get("decode_bytes_per_launch"),
+                         "peak_kind": f"{pk} copy bandwidth", "bytes_per_launch": dbytes,
+                         "kernel_ms": dec_kernel_ms}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all")
+    ap.add_argument("--decode-steps", type=int, default=DECODE["steps"])
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gdn(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

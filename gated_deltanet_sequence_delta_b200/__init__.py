@@ -1,0 +1,18 @@
+"""Gated DeltaNet core (gated delta rule) for NVIDIA B200, sm_100a.
+
+The computation lives in ``libgdn.so`` (C ABI: ``include/gdn.h``); this package
+is its thin binding.  Names are re-exported lazily so that ``inputs`` (the
+seeded workload generator) can be imported without loading torch or the
+library.
+"""
+_BINDING = ("gdn_gates", "gdn_chunk_prefill", "gdn_chunk_prefill_status", "gdn_decode_step",
+            "GDNError", "GDNLibraryError", "prefill_workspace_bytes", "kernel_launches")
+
+__all__ = list(_BINDING)
+
+
+def __getattr__(name):
+    if name in _BINDING:
+        from . import binding
+        return getattr(binding, name)
+    raise AttributeError(name)

@@ -1,0 +1,205 @@
+"""Thin Python binding over the C ABI of ``include/gdn.h`` (``libgdn.so``).
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream; outputs
+that the caller does not pass are allocated here with ``torch.empty``.
+
+The library is loaded on first use.  If ``libgdn.so`` is missing or cannot be
+loaded, every call raises ``GDNLibraryError``: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "gdn.h")
+
+GDN_F32, GDN_BF16 = 0, 1
+STATUS_NAMES = {0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_ALIGN",
+                4: "GDN_ERR_UNSUPPORTED", 5: "GDN_ERR_ALIAS", 6: "GDN_ERR_WORKSPACE",
+                7: "GDN_ERR_CUDA", 8: "GDN_ERR_DEVICE"}
+
+
+class GDNLibraryError(RuntimeError):
+    pass
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+_i32, _i64, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+_SIGS = {
+    "gdn_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "gdn_abi_version": ([], ctypes.c_int),
+    "gdn_last_cuda_error": ([], ctypes.c_int),
+    "gdn_kernel_launches": ([], ctypes.c_uint64),
+    "gdn_gates": ([_vp, _vp, ctypes.c_int, _vp, _vp, _i64, _i32, _vp, _vp, _vp], ctypes.c_int),
+    "gdn_chunk_prefill_workspace_bytes": ([_i64, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int], _sz),
+    "gdn_chunk_prefill": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+                           _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "gdn_chunk_prefill_status": ([_vp, _vp, ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_decode_step": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                         _f32, _i32, _vp, _vp], ctypes.c_int),
+}
+
+_LIB = None
+
+
+def header_functions(path: str = HEADER) -> list[str]:
+    """Names of the functions ``include/gdn.h`` declares."""
+    src = open(path).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*GDN_API\b[^(;]*?\b(gdn_\w+)\s*\(", src, re.M)))
+
+
+def lib(path: str | None = None):
+    """The loaded library (raises GDNLibraryError if it is not built)."""
+    global _LIB
+    if _LIB is not None and path is None:
+        return _LIB
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise GDNLibraryError(
+            f"{p} is not built; run `python -m gated_deltanet_sequence_delta_b200.build`")
+    try:
+        L = ctypes.CDLL(p)
+    except OSError as e:  # pragma: no cover
+        raise GDNLibraryError(f"cannot load {p}: {e}") from e
+    for name, (argtypes, restype) in _SIGS.items():
+        fn = getattr(L, name)
+        fn.argtypes = argtypes
+        fn.restype = restype
+    if path is None:
+        _LIB = L
+    return L
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().gdn_kernel_launches())
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        name = lib().gdn_status_string(status).decode()
+        extra = ""
+        if status == 7:
+            extra = f" (cudaError {lib().gdn_last_cuda_error()})"
+        raise GDNError(status, f"{what}: {name}{extra}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+# ---------------------------------------------------------------------------
+def gdn_gates(a: torch.Tensor, b: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor,
+              g: torch.Tensor | None = None, beta: torch.Tensor | None = None):
+    """g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b).
+    a, b [..., HV] fp32/bf16; A_log, dt_bias [HV] fp32.  Returns fp32 (g, beta)."""
+    HV = A_log.shape[-1]
+    if a.shape != b.shape or a.shape[-1] != HV or a.dtype != b.dtype:
+        raise ValueError("a, b must share shape [..., HV] and dtype")
+    if A_log.dtype != torch.float32 or dt_bias.dtype != torch.float32:
+        raise TypeError("A_log, dt_bias must be fp32")
+    g = torch.empty(a.shape, dtype=torch.float32, device=a.device) if g is None else g
+    beta = torch.empty(a.shape, dtype=torch.float32, device=a.device) if beta is None else beta
+    n = a.numel() // HV
+    st = lib().gdn_gates(_ptr(a), _ptr(b), _dtype_code(a), _ptr(A_log), _ptr(dt_bias), n, HV,
+                         _ptr(g), _ptr(beta), _stream())
+    _check(st, "gdn_gates")
+    return g, beta
+
+
+def prefill_workspace_bytes(n_tokens, n_seqs, HK, HV, Dk, Dv, BT, io_dtype) -> int:
+    return int(lib().gdn_chunk_prefill_workspace_bytes(n_tokens, n_seqs, HK, HV, Dk, Dv, BT, io_dtype))
+
+
+def gdn_chunk_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, BT: int = 64,
+                      scale: float = 1.0, qk_l2norm: bool = True, output_final_state: bool = True,
+                      o=None, final_state=None, workspace=None):
+    """Chunked prefill.  Dense: q, k [B, T, HK, Dk], v [B, T, HV, Dv], g, beta [B, T, HV].
+    Packed: B = 1 and cu_seqlens int32 [N + 1].  Returns (o, final_state or None)."""
+    B, T, HK, Dk = q.shape
+    HV, Dv = v.shape[-2:]
+    if k.shape != q.shape or v.shape[:2] != (B, T) or g.shape != (B, T, HV) or beta.shape != g.shape:
+        raise ValueError("inconsistent q/k/v/g/beta shapes")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    if g.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("g, beta must be fp32")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    dcode = _dtype_code(q)
+    if o is None:
+        o = torch.empty((B, T, HV, Dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, HV, Dk, Dv), dtype=torch.float32, device=q.device)
+    need = prefill_workspace_bytes(B * T, N, HK, HV, Dk, Dv, BT, dcode)
+    if need == 0:
+        _check(4, "gdn_chunk_prefill")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().gdn_chunk_prefill(
+        _ptr(q), _ptr(k), _ptr(v), dcode, _ptr(g), _ptr(beta), _ptr(initial_state),
+        _ptr(cu_seqlens), B, T, N, HK, HV, Dk, Dv, BT, float(scale), int(bool(qk_l2norm)),
+        _ptr(o), _ptr(final_state), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, "gdn_chunk_prefill")
+    return o, final_state
+
+
+def gdn_chunk_prefill_status(workspace: torch.Tensor) -> int:
+    """Synchronise the current stream and return the workspace's device error word."""
+    word = _i32(0)
+    st = lib().gdn_chunk_prefill_status(_ptr(workspace), _stream(), ctypes.byref(word))
+    if st not in (0, 8):
+        _check(st, "gdn_chunk_prefill_status")
+    return int(word.value)
+
+
+def gdn_decode_step(q, k, v, g, beta, state, scale: float = 1.0, qk_l2norm: bool = True, o=None):
+    """One token per sequence: q, k [B, HK, Dk]; v [B, HV, Dv]; g, beta [B, HV] fp32;
+    state [B, HV, Dk, Dv] fp32 updated in place.  Returns o [B, HV, Dv]."""
+    B, HK, Dk = q.shape
+    HV, Dv = v.shape[-2:]
+    if k.shape != q.shape or v.shape[0] != B or g.shape != (B, HV) or beta.shape != (B, HV):
+        raise ValueError("inconsistent decode shapes")
+    if state.shape != (B, HV, Dk, Dv) or state.dtype != torch.float32:
+        raise ValueError("state must be fp32 [B, HV, Dk, Dv]")
+    if o is None:
+        o = torch.empty((B, HV, Dv), dtype=q.dtype, device=q.device)
+    st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta),
+                               _ptr(state), B, HK, HV, Dk, Dv, float(scale), int(bool(qk_l2norm)),
+                               _ptr(o), _stream())
+    _check(st, "gdn_decode_step")
+    return o

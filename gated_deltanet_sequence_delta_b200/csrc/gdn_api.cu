@@ -1,0 +1,199 @@
+// gdn_api.cu -- the C ABI declared in gdn.h: host-side validation, then launches.
+// Nothing is launched unless every check passes; nothing is allocated or freed.
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "gdn.h"
+#include "gdn_internal.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+std::atomic<uint64_t> g_launches{0};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+    const void* p;
+    size_t bytes;
+};
+
+bool overlap(Range a, Range b) {
+    if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+    return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+size_t esize(gdn_dtype d) { return d == GDN_BF16 ? 2 : 4; }
+bool dtype_ok(gdn_dtype d) { return d == GDN_F32 || d == GDN_BF16; }
+bool head_dim_ok(int32_t d) { return d == 64 || d == 128; }
+
+gdn_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return GDN_OK;
+    g_last_cuda_error = (int)e;
+    return GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+namespace gdn {
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace gdn
+
+extern "C" {
+
+uint64_t gdn_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* gdn_status_string(int status) {
+    switch (status) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_NULL: return "GDN_ERR_NULL: a required pointer is NULL";
+        case GDN_ERR_SHAPE: return "GDN_ERR_SHAPE: a size is out of range or inconsistent";
+        case GDN_ERR_ALIGN: return "GDN_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: head dim, chunk size or dtype not implemented";
+        case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS: an output overlaps an input or another output";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA call or launch failed";
+        case GDN_ERR_DEVICE: return "GDN_ERR_DEVICE: a device-side check failed";
+        default: return "GDN: unknown status";
+    }
+}
+
+int gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+int gdn_last_cuda_error(void) { return g_last_cuda_error; }
+
+gdn_status gdn_gates(const void* a, const void* b, gdn_dtype ab_dtype, const float* A_log,
+                     const float* dt_bias, int64_t n_tokens, int32_t HV, float* g, float* beta,
+                     void* stream) {
+    if (!A_log || !dt_bias) return GDN_ERR_NULL;
+    if (HV <= 0 || n_tokens < 0) return GDN_ERR_SHAPE;
+    if (!dtype_ok(ab_dtype)) return GDN_ERR_UNSUPPORTED;
+    if (n_tokens == 0) return GDN_OK;
+    if (!a || !b || !g || !beta) return GDN_ERR_NULL;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(g) || !aligned16(beta) || !aligned16(A_log) ||
+        !aligned16(dt_bias))
+        return GDN_ERR_ALIGN;
+    const size_t n = (size_t)n_tokens * (size_t)HV;
+    const Range ra{a, n * esize(ab_dtype)}, rb{b, n * esize(ab_dtype)};
+    const Range rA{A_log, (size_t)HV * 4}, rd{dt_bias, (size_t)HV * 4};
+    const Range rg{g, n * 4}, rbeta{beta, n * 4};
+    for (Range out : {rg, rbeta})
+        for (Range in : {ra, rb, rA, rd})
+            if (overlap(out, in)) return GDN_ERR_ALIAS;
+    if (overlap(rg, rbeta)) return GDN_ERR_ALIAS;
+    return cuda_status(gdn::launch_gates(a, b, ab_dtype == GDN_BF16, A_log, dt_bias, n_tokens, HV,
+                                         g, beta, (cudaStream_t)stream));
+}
+
+size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seqs, int32_t HK, int32_t HV,
+                                         int32_t Dk, int32_t Dv, int32_t BT, gdn_dtype io_dtype) {
+    if (n_tokens < 0 || n_seqs < 0 || HK <= 0 || HV <= 0 || HV % HK != 0) return 0;
+    if (!head_dim_ok(Dk) || !head_dim_ok(Dv) || !dtype_ok(io_dtype)) return 0;
+    if (!(BT == 16 || BT == 32 || BT == 64)) return 0;
+    if (io_dtype == GDN_BF16 && BT != 64) return 0;
+    return gdn::kStatusBytes;
+}
+
+gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                             const float* g, const float* beta, const float* initial_state,
+                             const int32_t* cu_seqlens, int32_t B, int64_t T, int32_t n_seqs,
+                             int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
+                             float scale, int32_t qk_l2norm, void* o, float* final_state,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    // ---- sizes -----------------------------------------------------------------
+    if (B < 0 || T < 0 || n_seqs < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || BT <= 0)
+        return GDN_ERR_SHAPE;
+    if (HV % HK != 0) return GDN_ERR_SHAPE;
+    if (cu_seqlens) {
+        if (B != 1) return GDN_ERR_SHAPE;
+        if (T > INT32_MAX) return GDN_ERR_SHAPE;
+    } else if (n_seqs != B) {
+        return GDN_ERR_SHAPE;
+    }
+    if (!dtype_ok(io_dtype) || !head_dim_ok(Dk) || !head_dim_ok(Dv)) return GDN_ERR_UNSUPPORTED;
+    const size_t need = gdn_chunk_prefill_workspace_bytes((int64_t)B * T, n_seqs, HK, HV, Dk, Dv,
+                                                          BT, io_dtype);
+    if (need == 0) return GDN_ERR_UNSUPPORTED;
+    const int64_t n_tok = (int64_t)B * T;
+    if (n_seqs == 0) return GDN_OK;
+    // ---- pointers ----------------------------------------------------------------
+    if (!workspace) return GDN_ERR_WORKSPACE;
+    if (workspace_bytes < need) return GDN_ERR_WORKSPACE;
+    if (n_tok > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
+    if (cu_seqlens == nullptr && n_tok == 0 && final_state == nullptr) return GDN_OK;
+    const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    // ---- aliasing ----------------------------------------------------------------
+    const size_t es = esize(io_dtype);
+    const size_t state_bytes = (size_t)n_seqs * HV * Dk * Dv * 4;
+    const Range rq{q, (size_t)n_tok * HK * Dk * es}, rk{k, (size_t)n_tok * HK * Dk * es};
+    const Range rv{v, (size_t)n_tok * HV * Dv * es};
+    const Range rg{g, (size_t)n_tok * HV * 4}, rb{beta, (size_t)n_tok * HV * 4};
+    const Range rh0{initial_state, state_bytes}, rcu{cu_seqlens, cu_seqlens ? (size_t)(n_seqs + 1) * 4 : 0};
+    const Range ro{o, (size_t)n_tok * HV * Dv * es}, rhT{final_state, state_bytes};
+    const Range rws{workspace, workspace_bytes};
+    for (Range out : {ro, rhT, rws}) {
+        for (Range in : {rq, rk, rv, rg, rb, rcu})
+            if (overlap(out, in)) return GDN_ERR_ALIAS;
+    }
+    if (overlap(ro, rhT) || overlap(ro, rws) || overlap(rhT, rws) || overlap(ro, rh0) ||
+        overlap(rws, rh0))
+        return GDN_ERR_ALIAS;
+    // final_state may be exactly initial_state (in-place carry), nothing else
+    if (overlap(rhT, rh0) && final_state != initial_state) return GDN_ERR_ALIAS;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t* status = reinterpret_cast<int32_t*>(workspace);
+    gdn_status st = cuda_status(gdn::launch_check_cu_seqlens(cu_seqlens, n_seqs, T, status, s));
+    if (st != GDN_OK) return st;
+
+    gdn::PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.bf16 = io_dtype == GDN_BF16;
+    a.g = g; a.beta = beta; a.h0 = initial_state; a.cu = cu_seqlens;
+    a.T = T; a.n_seqs = n_seqs; a.HK = HK; a.HV = HV; a.Dk = Dk; a.Dv = Dv; a.BT = BT;
+    a.scale = scale; a.l2norm = qk_l2norm ? 1 : 0; a.o = o; a.hT = final_state;
+    a.status = status;
+    a.scratch = static_cast<char*>(workspace) + gdn::kStatusBytes;
+    a.scratch_bytes = workspace_bytes - gdn::kStatusBytes;
+    return cuda_status(gdn::launch_prefill_cudacore(a, s));
+}
+
+gdn_status gdn_chunk_prefill_status(const void* workspace, void* stream, int32_t* device_error) {
+    if (!workspace || !device_error) return GDN_ERR_NULL;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e);
+    int32_t word = 0;
+    e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    *device_error = word;
+    return word ? GDN_ERR_DEVICE : GDN_OK;
+}
+
+gdn_status gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                           const float* g, const float* beta, float* state, int32_t B, int32_t HK,
+                           int32_t HV, int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm,
+                           void* o, void* stream) {
+    if (B < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || HV % HK != 0) return GDN_ERR_SHAPE;
+    if (!dtype_ok(io_dtype) || !head_dim_ok(Dk) || !head_dim_ok(Dv)) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_NULL;
+    const void* ptrs[] = {q, k, v, g, beta, state, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t es = esize(io_dtype);
+    const Range rq{q, (size_t)B * HK * Dk * es}, rk{k, (size_t)B * HK * Dk * es};
+    const Range rv{v, (size_t)B * HV * Dv * es}, rg{g, (size_t)B * HV * 4}, rb{beta, (size_t)B * HV * 4};
+    const Range rs{state, (size_t)B * HV * Dk * Dv * 4}, ro{o, (size_t)B * HV * Dv * es};
+    for (Range out : {rs, ro})
+        for (Range in : {rq, rk, rv, rg, rb})
+            if (overlap(out, in)) return GDN_ERR_ALIAS;
+    if (overlap(rs, ro)) return GDN_ERR_ALIAS;
+    return cuda_status(gdn::launch_decode(q, k, v, io_dtype == GDN_BF16, g, beta, state, B, HK, HV,
+                                          Dk, Dv, scale, qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// gdn_internal.cuh -- private declarations shared by the library's .cu files.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+// ---- element access ------------------------------------------------------
+__device__ __forceinline__ float load_elem(const float* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p, int64_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_elem(float* p, int64_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, int64_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// softplus(x) = log(1 + e^x) in the overflow-free form max(x,0) + log1p(e^{-|x|}).
+__device__ __forceinline__ float softplus_f(float x) {
+    return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+}
+
+// L2-normalisation factor 1 / sqrt(sum x^2 + 1e-6) (flag off: 1).
+__device__ __forceinline__ float l2_inv(float sumsq, int enabled) {
+    return enabled ? 1.0f / sqrtf(sumsq + 1e-6f) : 1.0f;
+}
+
+// Launch accounting: every launcher calls count_launch() after a successful launch.
+void count_launch(int n = 1);
+
+// Workspace layout: [0, 256) status words; then kernel-specific scratch.
+constexpr size_t kStatusBytes = 256;
+
+// ---- launchers (return cudaError_t of the launch) -------------------------
+cudaError_t launch_gates(const void* a, const void* b, bool ab_bf16, const float* A_log,
+                         const float* dt_bias, int64_t n_tokens, int HV, float* g, float* beta,
+                         cudaStream_t s);
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16,
+                          const float* g, const float* beta, float* state, int B, int HK,
+                          int HV, int Dk, int Dv, float scale, int l2norm, void* o,
+                          cudaStream_t s);
+
+struct PrefillArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    bool bf16;
+    const float* g;
+    const float* beta;
+    const float* h0;          // may be null
+    const int32_t* cu;        // may be null (dense)
+    int64_t T;                // tokens per sequence (dense) or total (packed)
+    int n_seqs, HK, HV, Dk, Dv, BT;
+    float scale;
+    int l2norm;
+    void* o;
+    float* hT;                // may be null
+    int32_t* status;          // device status word (workspace)
+    void* scratch;            // workspace after the status words
+    size_t scratch_bytes;
+};
+
+cudaError_t launch_check_cu_seqlens(const int32_t* cu, int n_seqs, int64_t T, int32_t* status,
+                                    cudaStream_t s);
+cudaError_t launch_prefill_cudacore(const PrefillArgs& a, cudaStream_t s);
+
+}  // namespace gdn

@@ -1,0 +1,177 @@
+/*
+ * gdn.h -- C ABI of the Gated DeltaNet core for NVIDIA B200 (sm_100a).
+ *
+ * The library computes the gated delta rule in two modes, chunked prefill and
+ * a one-token recurrent decode step, plus the gate computation that feeds both.
+ *
+ *   Gates ("Gated DeltaNet ... Qwen3-next" page, section 2.1, gate code):
+ *       beta = sigmoid(b),  g = -exp(A_log) * softplus(a + dt_bias),  alpha = exp(g)
+ *   Rule ("Gated DeltaNet and reasoning scaffolds" research log, third update rule):
+ *       S_t = S_{t-1} (alpha_t (I - beta_t k_t k_t^T)) + beta_t v_t k_t^T,  o_t = scale * S_t q_t
+ *
+ * State orientation.  S_t is Dv x Dk (S k ~ v).  The library stores its
+ * transpose H = S^T, shape [.., Dk, Dv] row-major (the "k delta^T" form of the
+ * "QWEN3.5" Q&A page, question 2), always in fp32: one 128 x 128 head is 64 KB.
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE memory, allocated, owned and freed by the
+ *     caller.  The library never allocates, frees or synchronises, except in
+ *     gdn_chunk_prefill_status(), which synchronises the given stream.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Arguments are validated on the host before anything is
+ *     launched; a non-GDN_OK return means nothing was launched.
+ *   - Tensors are contiguous, token-major:  q, k [.., HK, Dk];  v, o [.., HV, Dv];
+ *     g, beta [.., HV].  Value head h reads q/k head h / (HV / HK).
+ *   - Pointers must be 16-byte aligned.  Outputs must not overlap any input or
+ *     each other (checked by address range).
+ *   - Supported sizes: Dk, Dv in {64, 128}; HV % HK == 0.
+ *   - io dtype GDN_BF16: q, k, v, o are bf16 and all arithmetic on them is fp32
+ *     accumulation with bf16 tensor-core operands; GDN_F32: everything fp32 on
+ *     CUDA cores (no TF32).
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_NULL = 1,        /* a required pointer is NULL                                  */
+    GDN_ERR_SHAPE = 2,       /* a size is negative, zero where it must not be, or inconsistent */
+    GDN_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                            */
+    GDN_ERR_UNSUPPORTED = 4, /* valid but not implemented (head dim, chunk size, dtype)     */
+    GDN_ERR_ALIAS = 5,       /* an output overlaps an input or another output               */
+    GDN_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than the size query returned      */
+    GDN_ERR_CUDA = 7,        /* a CUDA call or launch failed                                */
+    GDN_ERR_DEVICE = 8       /* a device-side check failed (reported by a status query)     */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Device-side error codes written into the prefill workspace's status word. */
+#define GDN_DEVERR_NONE 0
+#define GDN_DEVERR_CU_SEQLENS 1   /* cu_seqlens[0] != 0, decreasing, or last != T */
+
+/* Human-readable name of a gdn_status value (static storage, never NULL). */
+GDN_API const char* gdn_status_string(int status);
+
+/* GDN_ABI_VERSION of the loaded library. */
+GDN_API int gdn_abi_version(void);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all threads), counted at each successful launch.  For accounting only. */
+GDN_API uint64_t gdn_kernel_launches(void);
+
+/* Last CUDA error code (cudaError_t as int) seen by a call that returned
+ * GDN_ERR_CUDA on this host thread; 0 if none. */
+GDN_API int gdn_last_cuda_error(void);
+
+/*
+ * gdn_gates -- the gate formula ("Gated DeltaNet ... Qwen3-next" page, section 2.1).
+ *   a, b      [n_tokens, HV]  fp32 or bf16 (ab_dtype)       (read)
+ *   A_log     [HV] fp32,  dt_bias [HV] fp32                  (read)
+ *   g, beta   [n_tokens, HV] fp32                            (written)
+ *   g = -exp(A_log[h]) * softplus(a[t,h] + dt_bias[h]);  beta = 1 / (1 + exp(-b[t,h])).
+ * n_tokens may be 0 (nothing launched).  Errors: NULL, SHAPE (HV <= 0 or
+ * n_tokens < 0), ALIGN, ALIAS (g/beta overlapping inputs or each other), CUDA.
+ */
+GDN_API gdn_status gdn_gates(const void* a, const void* b, gdn_dtype ab_dtype,
+                     const float* A_log, const float* dt_bias,
+                     int64_t n_tokens, int32_t HV,
+                     float* g, float* beta, void* stream);
+
+/*
+ * Workspace size in bytes that gdn_chunk_prefill needs for these sizes (always
+ * >= 256: the first 256 bytes hold the device status word).  Returns 0 for
+ * sizes that gdn_chunk_prefill would reject.
+ */
+GDN_API size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seqs,
+                                         int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                                         int32_t BT, gdn_dtype io_dtype);
+
+/*
+ * gdn_chunk_prefill -- the rule over whole sequences, computed chunk by chunk
+ * ("QWEN3.5" Q&A page, question 1: chunks of BT tokens, parallel inside a chunk,
+ * state carried serially across chunks; the call shape is the
+ * chunk_gated_delta_rule(query, key, value, g, beta, initial_state) ->
+ * (out, last_state) call of the "Gated DeltaNet ... Qwen3-next" page, section 3.1).
+ *
+ *   Dense layout (cu_seqlens == NULL): B sequences of T tokens each; n_seqs must
+ *   equal B.  Packed layout (cu_seqlens != NULL): B must be 1, T is the total
+ *   token count, and sequence n is tokens cu_seqlens[n] .. cu_seqlens[n+1]-1.
+ *
+ *   q, k          [B, T, HK, Dk]   io_dtype                  (read)
+ *   v             [B, T, HV, Dv]   io_dtype                  (read)
+ *   g, beta       [B, T, HV]       fp32 log-decay and write strength (read)
+ *   initial_state [n_seqs, HV, Dk, Dv] fp32, or NULL for zero states (read)
+ *   cu_seqlens    [n_seqs + 1] int32 device, or NULL          (read)
+ *   o             [B, T, HV, Dv]   io_dtype                  (written)
+ *   final_state   [n_seqs, HV, Dk, Dv] fp32, or NULL          (written; may
+ *                 equal initial_state exactly for an in-place update, no other
+ *                 overlap allowed)
+ *   workspace     device scratch of >= gdn_chunk_prefill_workspace_bytes(...) bytes,
+ *                 owned by the caller, contents need not be initialised; it must
+ *                 not be shared by calls that may run concurrently.
+ *   BT            chunk length: 64 (GDN_BF16) or 16, 32, 64 (GDN_F32).  BT only
+ *                 changes rounding, never the result's definition.
+ *   scale         multiplies o (1.0 = the plain rule).
+ *   qk_l2norm     nonzero: q and k rows are replaced by x / sqrt(sum x^2 + 1e-6)
+ *                 before use (per token and q/k head).
+ *
+ * cu_seqlens is checked on the device (first entry 0, non-decreasing, last
+ * entry T).  A bad table makes every kernel of the call exit without writing o
+ * or final_state and leaves GDN_DEVERR_CU_SEQLENS in the workspace status word;
+ * read it with gdn_chunk_prefill_status().  Zero-length sequences are allowed
+ * (their final state equals the initial state).
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, ALIAS, WORKSPACE, CUDA.
+ */
+GDN_API gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                             const float* g, const float* beta,
+                             const float* initial_state, const int32_t* cu_seqlens,
+                             int32_t B, int64_t T, int32_t n_seqs,
+                             int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                             int32_t BT, float scale, int32_t qk_l2norm,
+                             void* o, float* final_state,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads the device status word of a prefill
+ * workspace into *device_error (GDN_DEVERR_*).  Returns GDN_ERR_DEVICE if it
+ * is nonzero, GDN_ERR_CUDA if the synchronisation failed, else GDN_OK.
+ */
+GDN_API gdn_status gdn_chunk_prefill_status(const void* workspace, void* stream, int32_t* device_error);
+
+/*
+ * gdn_decode_step -- one token per sequence, state updated in place (the
+ * incremental update of the "QWEN3.5" Q&A page, question 2a: decay the whole
+ * state by alpha, then clear and write along the current key with strength beta).
+ *   q, k   [B, HK, Dk] io_dtype;  v [B, HV, Dv] io_dtype;  g, beta [B, HV] fp32  (read)
+ *   state  [B, HV, Dk, Dv] fp32                            (read and written in place)
+ *   o      [B, HV, Dv] io_dtype                            (written; o = scale * S_t q_t
+ *                                                           with the updated state)
+ * B may be 0 (nothing launched).
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, ALIAS, CUDA.
+ */
+GDN_API gdn_status gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                           const float* g, const float* beta, float* state,
+                           int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                           float scale, int32_t qk_l2norm, void* o, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,146 @@
+"""Shared test harness: run a seeded workload through the CUDA library (via the C
+ABI binding) and through the CPU oracle, and compare them.
+
+Tolerances (the bar every GPU parity test uses):
+  * bf16 q/k/v with fp32 state: max |x_gpu - x_ref| <= 2e-2 * RMS(x_ref)
+  * fp32 mode:                  max |x_gpu - x_ref| <= 1e-4 * RMS(x_ref)
+applied to the outputs o and to the final states, separately.
+
+bf16 outputs.  Rounding the exact result to bf16 (round to nearest) moves an
+element x by up to 2^-8 |x|.  In these workloads max|o| is 8-10 times RMS(o), so
+that rounding alone can exceed 2e-2 * RMS(o) even for a perfect kernel.  For a
+bf16 output the bound is therefore applied to the arithmetic:
+    |o_gpu - o_ref| <= tol * RMS(o_ref) + 2^-8 |o_ref|      (elementwise)
+the second term being the representation bound of the output format.  fp32
+outputs and the (always fp32) final states take the bound as stated.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from gated_deltanet_sequence_delta_b200 import inputs as I
+
+TOL = {I.BF16: 2e-2, I.F32: 1e-4}
+
+
+def rms_err(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    assert np.all(np.isfinite(got)), "non-finite values in GPU result"
+    return err, rms
+
+
+BF16_REP = 2.0 ** -8   # relative representation bound of round-to-nearest bf16
+
+
+def assert_close(got, ref, tol, what="", out_bf16=False):
+    """max|got - ref| <= tol * RMS(ref) (plus 2^-8 |ref| per element when ``got``
+    was rounded to bf16).  Returns the arithmetic error relative to RMS(ref)."""
+    err, rms = rms_err(got, ref)
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if ref.size == 0:
+        return 0.0
+    excess = np.abs(got - ref) - (BF16_REP * np.abs(ref) if out_bf16 else 0.0)
+    arith = float(max(np.max(excess), 0.0))
+    assert arith <= tol * max(rms, 1e-30), (
+        f"{what}: max|err| {err:.3e} (beyond output rounding {arith:.3e}) > {tol:g} * RMS {rms:.3e}")
+    return arith / max(rms, 1e-30)
+
+
+# ---------------------------------------------------------------------------
+# device side
+# ---------------------------------------------------------------------------
+def to_dev(t, device="cuda"):
+    import torch
+    if isinstance(t, I.Tensor):
+        if t.dtype == I.BF16:
+            return torch.from_numpy(np.ascontiguousarray(t.data).view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(t.data)).to(device)
+    return torch.from_numpy(np.ascontiguousarray(t)).to(device)
+
+
+def to_np(x):
+    import torch
+    return x.detach().to(torch.float64).cpu().numpy()
+
+
+def gpu_gates(inp):
+    import gated_deltanet_sequence_delta_b200 as G
+    a = to_dev(inp.a)
+    b = to_dev(inp.b)
+    g, beta = G.gdn_gates(a, b, to_dev(inp.A_log), to_dev(inp.dt_bias))
+    if inp.g_reset is not None:
+        import torch
+        mask = to_dev(inp.g_reset).view(inp.B, inp.T)
+        g[mask] = -20.0
+    return g, beta
+
+
+def gpu_prefill(inp, BT=None, with_state=True):
+    """Gates then chunked prefill on the GPU; returns device tensors (o, hT, g, beta)."""
+    import gated_deltanet_sequence_delta_b200 as G
+    g, beta = gpu_gates(inp)
+    o, hT = G.gdn_chunk_prefill(
+        to_dev(inp.q), to_dev(inp.k), to_dev(inp.v), g, beta,
+        initial_state=None if inp.h0 is None else to_dev(inp.h0),
+        cu_seqlens=None if inp.cu_seqlens is None else to_dev(inp.cu_seqlens),
+        BT=BT or inp.BT, scale=inp.scale, qk_l2norm=inp.l2norm, output_final_state=with_state)
+    return o, hT, g, beta
+
+
+# ---------------------------------------------------------------------------
+# oracle side
+# ---------------------------------------------------------------------------
+def oracle_gates(inp):
+    import oracle
+    g, beta = oracle.gates(inp.a.astype(np.float64), inp.b.astype(np.float64),
+                           inp.A_log.astype(np.float64), inp.dt_bias.astype(np.float64))
+    if inp.g_reset is not None:
+        g.reshape(-1, inp.HV)[inp.g_reset] = -20.0
+    return g, beta
+
+
+def oracle_prefill(inp, heads=None):
+    """Oracle o [B, T, len(heads), Dv] and hT [N, len(heads), Dk, Dv] for the given
+    value heads (all heads by default)."""
+    import oracle
+    heads = list(range(inp.HV)) if heads is None else list(heads)
+    G_ = inp.HV // inp.HK
+    g, beta = oracle_gates(inp)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.astype(np.int64)
+    os_, hs = [], []
+    for h in heads:
+        hk = h // G_
+        q = inp.q.f64((slice(None), slice(None), slice(hk, hk + 1)))
+        k = inp.k.f64((slice(None), slice(None), slice(hk, hk + 1)))
+        v = inp.v.f64((slice(None), slice(None), slice(h, h + 1)))
+        h0 = None if inp.h0 is None else inp.h0[:, h:h + 1].astype(np.float64)
+        gh = g[:, :, h:h + 1]
+        bh = beta[:, :, h:h + 1]
+        if cu is None:
+            o, hT = oracle.recurrence(q, k, v, gh, bh, h0=h0, scale=inp.scale, l2norm=inp.l2norm)
+        else:
+            o, hT = oracle.recurrence(q[0], k[0], v[0], gh[0], bh[0], h0=h0, cu_seqlens=cu,
+                                      scale=inp.scale, l2norm=inp.l2norm)
+            o = o[None]
+        os_.append(o)
+        hs.append(hT)
+    return np.concatenate(os_, axis=2), np.concatenate(hs, axis=1)
+
+
+def check_prefill(inp, heads=None, BT=None, tol=None):
+    """Run both sides and assert parity on o and the final state; returns the
+    relative errors (err / RMS) for o and state."""
+    tol = TOL[inp.io_dtype] if tol is None else tol
+    o, hT, _, _ = gpu_prefill(inp, BT=BT)
+    heads_l = list(range(inp.HV)) if heads is None else list(heads)
+    o_ref, h_ref = oracle_prefill(inp, heads_l)
+    o_g = to_np(o[:, :, heads_l])
+    h_g = to_np(hT[:, heads_l])
+    eo = assert_close(o_g, o_ref, tol, f"{inp.name}: o", out_bf16=inp.io_dtype == I.BF16)
+    eh = assert_close(h_g, h_ref, tol, f"{inp.name}: final state")
+    return eo, eh

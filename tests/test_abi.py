@@ -1,0 +1,110 @@
+"""The C-ABI library loads, exports what include/gdn.h declares, and rejects bad
+arguments on the host before launching anything (no GPU needed: every call here
+fails validation, or has nothing to do, before any CUDA call)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from gated_deltanet_sequence_delta_b200 import binding, build as gbuild
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return binding.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = binding.header_functions()
+    assert {"gdn_gates", "gdn_chunk_prefill", "gdn_decode_step"} <= set(names)
+    nm = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                        text=True, check=True).stdout
+    exported = {line.split()[-1] for line in nm.splitlines() if " T " in line}
+    for n in names:
+        assert n in exported, n
+        assert getattr(L, n) is not None
+    # nothing but the declared API is exported (hidden visibility elsewhere)
+    assert {e for e in exported if e.startswith("gdn")} == set(names)
+
+
+def test_version_and_strings(L):
+    assert L.gdn_abi_version() == 1
+    for s in range(9):
+        assert L.gdn_status_string(s).decode().startswith("GDN_")
+    assert b"unknown" in L.gdn_status_string(99)
+    assert L.gdn_last_cuda_error() == 0
+
+
+A = 0x7f0000000000          # fake, 16-byte aligned device addresses: never dereferenced
+MB = 1 << 20
+
+
+def _prefill(L, **kw):
+    args = dict(q=A, k=A + 64 * MB, v=A + 128 * MB, io=1, g=A + 192 * MB, beta=A + 200 * MB,
+                h0=None, cu=None, B=1, T=128, N=1, HK=2, HV=4, Dk=128, Dv=128, BT=64, scale=1.0,
+                l2=1, o=A + 256 * MB, hT=A + 384 * MB, ws=A + 448 * MB, ws_bytes=1 << 20)
+    args.update(kw)
+    return L.gdn_chunk_prefill(args["q"], args["k"], args["v"], args["io"], args["g"], args["beta"],
+                               args["h0"], args["cu"], args["B"], args["T"], args["N"], args["HK"],
+                               args["HV"], args["Dk"], args["Dv"], args["BT"], args["scale"],
+                               args["l2"], args["o"], args["hT"], args["ws"], args["ws_bytes"], None)
+
+
+def test_prefill_validation(L):
+    assert _prefill(L, q=None) == 1                       # NULL
+    assert _prefill(L, HV=3) == 2                         # HV % HK
+    assert _prefill(L, B=2, N=1) == 2                     # dense needs N == B
+    assert _prefill(L, cu=A + 500 * MB, B=2, N=2) == 2    # packed needs B == 1
+    assert _prefill(L, Dk=96) == 4                        # unsupported head dim
+    assert _prefill(L, BT=32) == 4                        # bf16 path needs BT = 64
+    assert _prefill(L, io=1, BT=128) == 4
+    assert _prefill(L, ws=None) == 6
+    assert _prefill(L, ws_bytes=16) == 6
+    assert _prefill(L, q=A + 8) == 3                      # misaligned
+    assert _prefill(L, o=A + 64) == 5                     # o overlaps q
+    assert _prefill(L, hT=A + 256 * MB + 4096) == 5       # final state overlaps o
+    assert _prefill(L, h0=A + 384 * MB + 64) == 5         # partial overlap of states
+    assert _prefill(L, N=0, B=0) == 0                     # nothing to do: no launch
+
+
+def test_prefill_workspace_query(L):
+    assert L.gdn_chunk_prefill_workspace_bytes(32768, 1, 16, 32, 128, 128, 64, 1) >= 256
+    assert L.gdn_chunk_prefill_workspace_bytes(256, 1, 2, 2, 64, 64, 64, 0) >= 256
+    assert L.gdn_chunk_prefill_workspace_bytes(256, 1, 2, 3, 64, 64, 64, 0) == 0
+    assert L.gdn_chunk_prefill_workspace_bytes(256, 1, 2, 2, 80, 64, 64, 0) == 0
+
+
+def test_gates_validation(L):
+    f = L.gdn_gates
+    assert f(A, A + MB, 0, None, A + 3 * MB, 10, 4, A + 4 * MB, A + 5 * MB, None) == 1
+    assert f(A, A + MB, 0, A + 2 * MB, A + 3 * MB, 10, 0, A + 4 * MB, A + 5 * MB, None) == 2
+    assert f(A, A + MB, 0, A + 2 * MB, A + 3 * MB, -1, 4, A + 4 * MB, A + 5 * MB, None) == 2
+    assert f(A, A + MB, 0, A + 2 * MB, A + 3 * MB, 10, 4, A + 16, A + 5 * MB, None) == 5
+    assert f(A, A + MB, 0, A + 2 * MB, A + 3 * MB, 10, 4, A + 4 * MB, A + 4 * MB + 16, None) == 5
+    assert f(A + 4, A + MB, 0, A + 2 * MB, A + 3 * MB, 10, 4, A + 4 * MB, A + 5 * MB, None) == 3
+    assert f(None, None, 0, A + 2 * MB, A + 3 * MB, 0, 4, None, None, None) == 0   # empty: no launch
+
+
+def test_decode_validation(L):
+    f = L.gdn_decode_step
+    base = [A, A + MB, A + 2 * MB, 1, A + 3 * MB, A + 4 * MB, A + 16 * MB, 4, 2, 4, 128, 128, 1.0, 1,
+            A + 8 * MB, None]
+    def call(**kw):
+        a = list(base)
+        for i, val in kw.items():
+            a[int(i[1:])] = val
+        return f(*a)
+    assert call(a6=None) == 1
+    assert call(a9=3) == 2
+    assert call(a10=32) == 4
+    assert call(a3=7) == 4
+    assert call(a14=A + 16 * MB + 128) == 5     # o inside the state
+    assert call(a6=A + 2 * MB) == 5             # state over v
+    assert call(a0=A + 2) == 3
+    assert call(a7=0) == 0                      # B = 0: nothing to do
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(binding.GDNLibraryError):
+        binding.lib(str(tmp_path / "nope.so"))
