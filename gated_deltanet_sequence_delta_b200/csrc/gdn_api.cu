@@ -93,6 +93,8 @@ size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seqs, int32
     if (!head_dim_ok(Dk) || !head_dim_ok(Dv) || !dtype_ok(io_dtype)) return 0;
     if (!(BT == 16 || BT == 32 || BT == 64)) return 0;
     if (io_dtype == GDN_BF16 && BT != 64) return 0;
+    if (io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT))
+        return gdn::prefill_tc_workspace_bytes(n_tokens, n_seqs, HK, HV);
     return gdn::kStatusBytes;
 }
 
@@ -147,8 +149,11 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dt
 
     cudaStream_t s = (cudaStream_t)stream;
     int32_t* status = reinterpret_cast<int32_t*>(workspace);
-    gdn_status st = cuda_status(gdn::launch_check_cu_seqlens(cu_seqlens, n_seqs, T, status, s));
-    if (st != GDN_OK) return st;
+    const bool use_tc = io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT);
+    if (!use_tc) {
+        gdn_status st = cuda_status(gdn::launch_check_cu_seqlens(cu_seqlens, n_seqs, T, status, s));
+        if (st != GDN_OK) return st;
+    }
 
     gdn::PrefillArgs a;
     a.q = q; a.k = k; a.v = v; a.bf16 = io_dtype == GDN_BF16;
@@ -158,6 +163,7 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dt
     a.status = status;
     a.scratch = static_cast<char*>(workspace) + gdn::kStatusBytes;
     a.scratch_bytes = workspace_bytes - gdn::kStatusBytes;
+    if (use_tc) return cuda_status(gdn::launch_prefill_tc(a, workspace, s));
     return cuda_status(gdn::launch_prefill_cudacore(a, s));
 }
 

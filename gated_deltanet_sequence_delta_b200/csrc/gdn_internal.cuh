@@ -75,4 +75,9 @@ cudaError_t launch_check_cu_seqlens(const int32_t* cu, int n_seqs, int64_t T, in
                                     cudaStream_t s);
 cudaError_t launch_prefill_cudacore(const PrefillArgs& a, cudaStream_t s);
 
+// Tensor-core (tcgen05) prefill: bf16, Dk = Dv = 128, BT = 64, HV / HK in {1, 2}.
+bool prefill_tc_supported(int Dk, int Dv, int HK, int HV, int BT);
+size_t prefill_tc_workspace_bytes(int64_t n_tokens, int n_seqs, int HK, int HV);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_t s);
+
 }  // namespace gdn

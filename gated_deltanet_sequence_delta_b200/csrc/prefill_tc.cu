@@ -1,0 +1,959 @@
+// prefill_tc.cu -- chunked prefill of the gated delta rule on the 5th-generation tensor
+// cores (tcgen05, TMA, TMEM), bf16 operands with fp32 accumulation and fp32 state.
+//
+// The chunk scheme ("QWEN3.5" Q&A page, question 1): time is cut into chunks of C = 64
+// tokens; inside a chunk the work is parallel, across chunks the state is carried
+// serially.  The chunk equations follow from the recurrence alone.  For one chunk of one
+// value head, with H0 = S^T (Dk x Dv) the state at the chunk start, raw (not yet
+// normalised) rows k_i, q_i, inverse norms rk_i, rq_i, write strengths b_i, and G_i the
+// running sum of the log-decays inside the chunk (gamma_i = exp(G_i)):
+//     L_ij = b_i exp(G_i - G_j) rk_i rk_j k_i.k_j   (i > j)      T = (I + L)^-1
+//     W    = T diag(b gamma rk) K,   U = T diag(b) V                     (chunk-local)
+//     P_ij = scale exp(G_i - G_j) rq_i rk_j q_i.k_j  (i >= j)
+//     Delta = U - W H0
+//     O     = diag(scale gamma rq) Q H0 + P Delta
+//     H_C   = gamma_C H0 + K^T diag(exp(G_C - G) rk) Delta
+// (with K_hat = diag(rk) K and Q_hat = diag(rq) Q the same reads diag(gamma) Q_hat H0 and
+// K_hat^T diag(exp(G_C - G)) Delta).
+// Every exponent evaluated is <= 0.
+//
+// Precision.  The output is a sum of terms much larger than itself (U - W H0 cancels, so
+// does P Delta against the decayed Q H0 part), so bf16 rounding of the intermediates
+// alone costs 3-5% of RMS(o).  Hence: the chunk-local products W and U are formed with
+// the T operands split into bf16 hi + lo parts against the exact bf16 inputs, and every
+// intermediate operand of the serial stage is fp16 (10-bit mantissa).  Data-dependent
+// operands (state, Delta, U) carry a power-of-two scale so fp16 range is never at issue.
+//
+// Two kernels:
+//  * chunk_prep (one CTA per chunk and q/k head, fully parallel): the Gram tiles
+//    [K;Q] K^T on tcgen05 (M=128), norms, gates, the unit-lower-triangular inverse T in
+//    fp32 on CUDA cores (16x16 diagonal blocks by substitution, off-diagonal blocks by
+//    block products), then W^T = K^T (T diag(b gamma rk))^T and U^T = V^T (T diag(b))^T on
+//    tcgen05 (M=128: Dk or Dv rows).  Writes fp16 W, U (scaled), P, the normalised fp16
+//    K_hat, Q_hat tiles and per-row scalars.
+//  * chunk_carry (one CTA per sequence, value head and 32-column slice of Dv; the value
+//    columns of the state evolve independently): walks the chunks in order.  Per chunk:
+//    [W;Q_hat] H0 (M=128) -> Delta on CUDA cores -> K_hat^T Delta~ and [0;P] Delta (M=128),
+//    state kept in fp32 registers, its scaled fp16 copy in shared memory as the next MMA
+//    operand.  A producer warp streams the operands through a 2-stage TMA ring.
+// All waits on mbarriers are bounded: on expiry the kernel records GDN_DEVERR_TIMEOUT in
+// the workspace status word and exits cleanly (TMEM freed).
+#include <cudaTypedefs.h>
+
+#include "gdn_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace gdn {
+namespace {
+
+using bf16 = __nv_bfloat16;
+using f16 = __half;
+constexpr int C = 64;      // chunk length
+constexpr int D = 128;     // head dim (Dk = Dv) of this path
+constexpr int NS = 32;     // value columns per carry CTA
+constexpr int NSTAGE = 2;  // TMA ring depth of the carry kernel
+constexpr int SC_FLOATS = 256;   // per (chunk, value head): a[64], d[64], scalars below
+constexpr int SC_GC = 128;       //   gamma_C = exp(G at the chunk's last token)
+constexpr int SC_UINV = 129;     //   U is stored as fp16(U * 2^-e); this holds 2^e
+constexpr int SC_VMAX = 130;     //   max |v| over the chunk's tile of this value head
+
+// power of two 2^e with max_abs * 2^-e in [0.5, 1) (1 for max_abs == 0 or non-finite)
+__device__ __forceinline__ float pow2_above(float max_abs) {
+    if (!(max_abs > 0.f) || !isfinite(max_abs)) return 1.f;
+    int e;
+    frexpf(max_abs, &e);
+    return ldexpf(1.f, e);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void record_timeout(int32_t* status) {
+    atomicCAS(status, GDN_DEVERR_NONE, GDN_DEVERR_TIMEOUT);
+}
+
+// true if any of the n threads meeting at barrier `id` passes pred = true
+__device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+// Locate chunk `chunk` of the flattened chunk list: its sequence n, first token s and
+// length cn.  chunk_off[n] is the first chunk of sequence n (chunk_off[N] = total).
+__device__ __forceinline__ bool locate_chunk(int chunk, const int32_t* __restrict__ chunk_off,
+                                             const int32_t* __restrict__ cu, int64_t T, int n_seqs,
+                                             int& n, int64_t& s, int& cn) {
+    if (chunk >= chunk_off[n_seqs]) return false;
+    int lo = 0, hi = n_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (chunk_off[mid] <= chunk) lo = mid; else hi = mid - 1;
+    }
+    n = lo;
+    const int64_t bos = cu ? (int64_t)cu[n] : (int64_t)n * T;
+    const int64_t len = cu ? (int64_t)cu[n + 1] - cu[n] : T;
+    const int j = chunk - chunk_off[n];
+    s = bos + (int64_t)C * j;
+    const int64_t rem = len - (int64_t)C * j;
+    cn = (int)(rem < C ? rem : C);
+    return cn > 0;
+}
+
+// ======================================================================================
+// chunk table: validate cu_seqlens (if any) and write chunk_off[0..N] (one CTA)
+// ======================================================================================
+__global__ void __launch_bounds__(1024) chunk_table_kernel(const int32_t* __restrict__ cu, int n_seqs,
+                                                           int64_t T, int32_t* __restrict__ chunk_off,
+                                                           int32_t* __restrict__ status) {
+    __shared__ int s_part[1024];
+    __shared__ int s_bad;
+    const int tid = threadIdx.x;
+    if (tid == 0) s_bad = 0;
+    __syncthreads();
+    const int per = (n_seqs + 1023) / 1024;
+    const int n0 = tid * per, n1 = min(n_seqs, n0 + per);
+    int local = 0;
+    for (int n = n0; n < n1; ++n) {
+        int64_t len = T;
+        if (cu) {
+            len = (int64_t)cu[n + 1] - cu[n];
+            if (len < 0) s_bad = 1;
+        }
+        if (len > 0) local += (int)((len + C - 1) / C);
+    }
+    if (cu && tid == 0 && (cu[0] != 0 || (int64_t)cu[n_seqs] != T)) s_bad = 1;
+    s_part[tid] = local;
+    __syncthreads();
+    // inclusive scan of the 1024 partial counts (Hillis-Steele)
+    for (int o = 1; o < 1024; o <<= 1) {
+        const int v = tid >= o ? s_part[tid - o] : 0;
+        __syncthreads();
+        s_part[tid] += v;
+        __syncthreads();
+    }
+    int off = s_part[tid] - local;
+    for (int n = n0; n < n1; ++n) {
+        chunk_off[n] = off;
+        int64_t len = cu ? (int64_t)cu[n + 1] - cu[n] : T;
+        if (len > 0) off += (int)((len + C - 1) / C);
+    }
+    if (tid == 1023) chunk_off[n_seqs] = s_part[1023];
+    __syncthreads();
+    if (tid == 0) *status = s_bad ? GDN_DEVERR_CU_SEQLENS : GDN_DEVERR_NONE;
+}
+
+// ======================================================================================
+// T = (I + L)^-1 for a 64 x 64 strictly lower L (fp32, row stride 65), 128 threads.
+// Writes the lower triangle of T including its unit diagonal; entries above the diagonal
+// are left untouched.  Blocks of 16: T_ii = (I + L_ii)^-1 by column substitution, then
+// T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj by increasing i - j.
+// ======================================================================================
+__device__ __forceinline__ void tinv64(const float (*L)[65], float (*Tm)[65], float (*X)[16][17], int tid) {
+    if (tid < 64) {
+        const int b = tid >> 4, c = tid & 15, o = 16 * b;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float acc = (i == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) acc = fmaf(-L[o + i][o + j], x[j], acc);
+            x[i] = acc;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (i >= c) Tm[o + i][o + c] = x[i];
+    }
+    __syncthreads();
+    // first sub-diagonal blocks (b+1, b), b = 0, 1, 2
+    for (int e = tid; e < 3 * 256; e += 128) {
+        const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
+        const int oi = 16 * (b + 1), oj = 16 * b;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if (k >= c) acc = fmaf(L[oi + r][oj + k], Tm[oj + k][oj + c], acc);
+        X[b][r][c] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < 3 * 256; e += 128) {
+        const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
+        const int oi = 16 * (b + 1), oj = 16 * b;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if (k <= r) acc = fmaf(Tm[oi + r][oi + k], X[b][k][c], acc);
+        Tm[oi + r][oj + c] = -acc;
+    }
+    __syncthreads();
+    // second sub-diagonal blocks (2, 0) and (3, 1)
+    for (int e = tid; e < 2 * 256; e += 128) {
+        const int p = e >> 8, r = (e >> 4) & 15, c = e & 15;
+        const int oi = 16 * (p + 2), oj = 16 * p, om = 16 * (p + 1);
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            if (k >= c) acc = fmaf(L[oi + r][oj + k], Tm[oj + k][oj + c], acc);
+            acc = fmaf(L[oi + r][om + k], Tm[om + k][oj + c], acc);
+        }
+        X[p][r][c] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < 2 * 256; e += 128) {
+        const int p = e >> 8, r = (e >> 4) & 15, c = e & 15;
+        const int oi = 16 * (p + 2), oj = 16 * p;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if (k <= r) acc = fmaf(Tm[oi + r][oi + k], X[p][k][c], acc);
+        Tm[oi + r][oj + c] = -acc;
+    }
+    __syncthreads();
+    // third sub-diagonal block (3, 0)
+    for (int e = tid; e < 256; e += 128) {
+        const int r = e >> 4, c = e & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            if (k >= c) acc = fmaf(L[48 + r][k], Tm[k][c], acc);
+            acc = fmaf(L[48 + r][16 + k], Tm[16 + k][c], acc);
+            acc = fmaf(L[48 + r][32 + k], Tm[32 + k][c], acc);
+        }
+        X[0][r][c] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < 256; e += 128) {
+        const int r = e >> 4, c = e & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if (k <= r) acc = fmaf(Tm[48 + r][48 + k], X[0][k][c], acc);
+        Tm[48 + r][c] = -acc;
+    }
+    __syncthreads();
+}
+
+// ======================================================================================
+// chunk_prep
+// ======================================================================================
+struct PrepSmem {
+    bf16 KQ[2][128 * 64];   // two 64-column halves of [K; Q] (rows 0-63 K, 64-127 Q), 16 KB each
+    bf16 V[2][64 * 64];     // two 64-column halves of V, 8 KB each
+    bf16 AW[64 * 64];       // hi part of T diag(b gamma rk), K-major B operand (rows i, K = j)
+    bf16 AU[64 * 64];       // hi part of T diag(b)
+    union {                 // L is dead once T is formed; its space then holds the lo parts
+        float L[64][65];
+        struct {
+            bf16 AWlo[64 * 64];
+            bf16 AUlo[64 * 64];
+        } lo;
+    } u;
+    float Tm[64][65];
+    float X[3][16][17];
+    float rk[64], rq[64], G[64], bt[64], bgr[64], red[8];
+    uint64_t bar_load, bar_v, bar_mma;
+    uint32_t tmem_base;
+};
+constexpr size_t kPrepSmemBytes = sizeof(PrepSmem) + 1024;
+constexpr uint32_t kPrepTmemCols = 256;
+
+template <int G>
+__global__ void __launch_bounds__(128, 2)
+chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                  const float* __restrict__ beta, const int32_t* __restrict__ cu,
+                  const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HV, float scale,
+                  int l2norm, int HK, f16* __restrict__ Wg, f16* __restrict__ Ug, f16* __restrict__ Pg,
+                  f16* __restrict__ QKg, float* __restrict__ SCg, int32_t* __restrict__ status) {
+    extern __shared__ uint8_t smem_raw[];
+    PrepSmem& S = *reinterpret_cast<PrepSmem*>(align1024(smem_raw));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int chunk = blockIdx.x, hk = blockIdx.y;
+    if (*reinterpret_cast<volatile int32_t*>(status) != 0) return;
+    int n, cn;
+    int64_t s;
+    if (!locate_chunk(chunk, chunk_off, cu, T, n_seqs, n, s, cn)) return;
+
+    if (warp == 0) {
+        tc::tmem_alloc(&S.tmem_base, kPrepTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (tid == 32) {
+        tc::mbar_init(&S.bar_load, 1);
+        tc::mbar_init(&S.bar_v, 1);
+        tc::mbar_init(&S.bar_mma, 1);
+        tc::fence_mbar_init();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t tD1 = tmem, tDW = tmem + 64, tDU = tmem + 128;
+    const int si = (int)s;
+
+    if (tid == 0) {
+        tc::mbar_expect_tx(&S.bar_load, 4 * 64 * 64 * 2);
+        tc::tma_load_3d(&S.KQ[0][0], &tm_k, &S.bar_load, 0, hk, si);
+        tc::tma_load_3d(&S.KQ[1][0], &tm_k, &S.bar_load, 64, hk, si);
+        tc::tma_load_3d(&S.KQ[0][64 * 64], &tm_q, &S.bar_load, 0, hk, si);
+        tc::tma_load_3d(&S.KQ[1][64 * 64], &tm_q, &S.bar_load, 64, hk, si);
+        tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+        tc::tma_load_3d(&S.V[0][0], &tm_v, &S.bar_v, 0, hk * G, si);
+        tc::tma_load_3d(&S.V[1][0], &tm_v, &S.bar_v, 64, hk * G, si);
+    }
+    bool ok = tc::mbar_wait(&S.bar_load, 0);
+    if (__syncthreads_or(!ok)) goto abort;
+
+    // ---- Gram tiles: D1[0:64] = K K^T, D1[64:128] = Q K^T (M=128, N=64, K=Dk) ---------
+    if (tid == 0) {
+        tc::tc_fence_after();
+        const uint32_t base = tc::smem_u32(&S.KQ[0][0]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t d = tc::desc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            tc::mma_bf16(tD1, d, d, tc::idesc_bf16(128, 64, 0, 0), kk > 0);
+        }
+        tc::mma_commit(&S.bar_mma);
+    }
+    if (tid >= 64) {   // inverse norms of q rows, from the raw tile (order inside a row is irrelevant)
+        float ss = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint4* row = reinterpret_cast<const uint4*>(&S.KQ[half][tid * 64]);
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16) {
+                const uint4 u = row[c16];
+                const bf16* e = reinterpret_cast<const bf16*>(&u);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const float x = __bfloat162float(e[t]);
+                    ss = fmaf(x, x, ss);
+                }
+            }
+        }
+        S.rq[tid - 64] = l2_inv(ss, l2norm);
+    }
+    ok = tc::mbar_wait(&S.bar_mma, 0);
+    if (__syncthreads_or(!ok)) goto abort;
+    tc::tc_fence_after();
+    {
+        float row[64];
+        tc::tmem_ld32(tD1 + lane_base, row);
+        tc::tmem_ld32(tD1 + lane_base + 32, row + 32);
+        tc::tmem_wait_ld();
+        if (tid < 64) {
+            float diag = 0.f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (j == tid) diag = row[j];
+            S.rk[tid] = l2_inv(diag, l2norm);   // k.k from the Gram diagonal
+        }
+        __syncthreads();
+        const float rki = tid < 64 ? S.rk[tid] : 0.f;
+        const float rqi = tid >= 64 ? S.rq[tid - 64] : 0.f;
+        {   // normalised fp16 copies of this row of K (tid < 64) or Q, in natural column order
+            const float rr = tid < 64 ? rki : rqi;
+            uint4* dst = reinterpret_cast<uint4*>(QKg + (((size_t)chunk * HK + hk) * 128 + tid) * D);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const uint4* row = reinterpret_cast<const uint4*>(&S.KQ[half][tid * 64]);
+#pragma unroll
+                for (int c16 = 0; c16 < 8; ++c16) {
+                    const uint4 u = row[c16 ^ (tid & 7)];   // logical chunk c16 sits at c16 ^ (row % 8)
+                    const bf16* e = reinterpret_cast<const bf16*>(&u);
+                    __align__(16) f16 hx[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) hx[t] = __float2half_rn(__bfloat162float(e[t]) * rr);
+                    dst[half * 8 + c16] = *reinterpret_cast<const uint4*>(hx);
+                }
+            }
+        }
+
+        for (int gi = 0; gi < G; ++gi) {
+            const int h = hk * G + gi;
+            const size_t ch = (size_t)chunk * HV + h;
+            // ---- gates of this value head: running sum of g, write strengths ---------
+            if (tid < 64) {
+                float gv = tid < cn ? g[(s + tid) * HV + h] : 0.f;
+                const float bv = tid < cn ? beta[(s + tid) * HV + h] : 0.f;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, gv, o);
+                    if ((tid & 31) >= o) gv += y;
+                }
+                S.G[tid] = gv;
+                S.bt[tid] = bv;
+            }
+            __syncthreads();
+            if (tid >= 32 && tid < 64) S.G[tid] += S.G[31];
+            __syncthreads();
+            if (tid < 64) S.bgr[tid] = S.bt[tid] * expf(S.G[tid]) * S.rk[tid];
+            const float Gl = S.G[63];   // padding adds 0, so this is G at the last token
+            // ---- L (strictly lower) and P (lower incl. diagonal), scalars -----------------
+            if (tid < 64) {
+                const int i = tid;
+                const float Gi = S.G[i], bi = S.bt[i] * rki;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    float v = 0.f;
+                    if (j < i && i < cn) v = bi * expf(Gi - S.G[j]) * S.rk[j] * row[j];
+                    S.u.L[i][j] = v;
+                }
+                SCg[ch * SC_FLOATS + 64 + i] = i < cn ? expf(Gl - Gi) : 0.f;
+            } else {
+                const int i = tid - 64;
+                const float Gi = S.G[i], qi = scale * rqi;
+                SCg[ch * SC_FLOATS + i] = i < cn ? scale * expf(Gi) : 0.f;
+                if (i == 0) SCg[ch * SC_FLOATS + SC_GC] = expf(Gl);
+                uint4* prow = reinterpret_cast<uint4*>(Pg + (ch * 64 + i) * 64);
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    __align__(16) f16 e[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        const int j = c8 * 8 + t;
+                        float v = 0.f;
+                        if (j <= i && i < cn) v = qi * expf(Gi - S.G[j]) * S.rk[j] * row[j];
+                        e[t] = __float2half_rn(v);
+                    }
+                    prow[c8] = *reinterpret_cast<const uint4*>(e);
+                }
+            }
+            __syncthreads();
+            tinv64(S.u.L, S.Tm, S.X, tid);
+            // ---- MMA operands T diag(b gamma rk) and T diag(b) as bf16 hi + lo parts ------
+            {
+                const int i = tid >> 1, c0 = (tid & 1) * 32;
+                uint8_t* aw = reinterpret_cast<uint8_t*>(S.AW);
+                uint8_t* au = reinterpret_cast<uint8_t*>(S.AU);
+                uint8_t* awl = reinterpret_cast<uint8_t*>(S.u.lo.AWlo);
+                uint8_t* aul = reinterpret_cast<uint8_t*>(S.u.lo.AUlo);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    __align__(16) bf16 w8[8], u8[8], wl8[8], ul8[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        const int j = c0 + cc * 8 + t;
+                        const float tij = j < i ? S.Tm[i][j] : (j == i ? 1.f : 0.f);
+                        const float wv = tij * S.bgr[j], uv = tij * S.bt[j];
+                        w8[t] = __float2bfloat16_rn(wv);
+                        u8[t] = __float2bfloat16_rn(uv);
+                        wl8[t] = __float2bfloat16_rn(wv - __bfloat162float(w8[t]));
+                        ul8[t] = __float2bfloat16_rn(uv - __bfloat162float(u8[t]));
+                    }
+                    const uint32_t off = tc::sw128_off(i, c0 + cc * 8);
+                    *reinterpret_cast<uint4*>(aw + off) = *reinterpret_cast<const uint4*>(w8);
+                    *reinterpret_cast<uint4*>(au + off) = *reinterpret_cast<const uint4*>(u8);
+                    *reinterpret_cast<uint4*>(awl + off) = *reinterpret_cast<const uint4*>(wl8);
+                    *reinterpret_cast<uint4*>(aul + off) = *reinterpret_cast<const uint4*>(ul8);
+                }
+            }
+            tc::fence_async_smem();
+            ok = tc::mbar_wait(&S.bar_v, gi & 1);
+            if (__syncthreads_or(!ok)) goto abort;
+            float vmax = 0.f;   // max |v| over the tile (rows past the chunk are masked out)
+            {
+                const int r = tid >> 1;
+                if (r < cn) {
+                    const uint4* vr = reinterpret_cast<const uint4*>(&S.V[tid & 1][r * 64]);
+#pragma unroll
+                    for (int c16 = 0; c16 < 8; ++c16) {
+                        const uint4 u = vr[c16];
+                        const bf16* e = reinterpret_cast<const bf16*>(&u);
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) vmax = fmaxf(vmax, fabsf(__bfloat162float(e[t])));
+                    }
+                }
+            }
+            // ---- W^T = K^T AW^T and U^T = V^T AU^T (M=128, N=64, K=64 tokens) -----------
+            if (tid == 0) {
+                tc::tc_fence_after();
+                const uint32_t kb = tc::smem_u32(&S.KQ[0][0]);
+                const uint32_t vb = tc::smem_u32(&S.V[0][0]);
+                const uint32_t awb = tc::smem_u32(S.AW), aub = tc::smem_u32(S.AU);
+                const uint32_t awl = tc::smem_u32(S.u.lo.AWlo), aul = tc::smem_u32(S.u.lo.AUlo);
+                constexpr uint32_t idx = tc::idesc_bf16(128, 64, 1, 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tDW, tc::desc_sw128(kb + kk * 2048, 16384, 1024),
+                                 tc::desc_sw128(awb + kk * 32, 16, 1024), idx, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tDW, tc::desc_sw128(kb + kk * 2048, 16384, 1024),
+                                 tc::desc_sw128(awl + kk * 32, 16, 1024), idx, 1);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tDU, tc::desc_sw128(vb + kk * 2048, 8192, 1024),
+                                 tc::desc_sw128(aub + kk * 32, 16, 1024), idx, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tDU, tc::desc_sw128(vb + kk * 2048, 8192, 1024),
+                                 tc::desc_sw128(aul + kk * 32, 16, 1024), idx, 1);
+                tc::mma_commit(&S.bar_mma);
+            }
+            ok = tc::mbar_wait(&S.bar_mma, (gi + 1) & 1);
+            if (__syncthreads_or(!ok)) goto abort;
+            tc::tc_fence_after();
+            if (tid == 0 && gi + 1 < G) {   // V buffer is free again: fetch the next head's V
+                tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+                tc::tma_load_3d(&S.V[0][0], &tm_v, &S.bar_v, 0, h + 1, si);
+                tc::tma_load_3d(&S.V[1][0], &tm_v, &S.bar_v, 64, h + 1, si);
+            }
+            // ---- epilogue: lane t of D_W / D_U is column t of W / U ----------------------
+            {
+                float w[64];
+                tc::tmem_ld32(tDW + lane_base, w);
+                tc::tmem_ld32(tDW + lane_base + 32, w + 32);
+                tc::tmem_wait_ld();
+                f16* Wd = Wg + ch * 64 * D + tid;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) Wd[i * D] = __float2half_rn(w[i]);
+                tc::tmem_ld32(tDU + lane_base, w);
+                tc::tmem_ld32(tDU + lane_base + 32, w + 32);
+                tc::tmem_wait_ld();
+                float umax = 0.f;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) umax = fmaxf(umax, fabsf(w[i]));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    umax = fmaxf(umax, __shfl_xor_sync(0xffffffffu, umax, o));
+                    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+                }
+                if ((tid & 31) == 0) {
+                    S.red[warp] = umax;
+                    S.red[4 + warp] = vmax;
+                }
+                __syncthreads();
+                umax = fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3]));
+                vmax = fmaxf(fmaxf(S.red[4], S.red[5]), fmaxf(S.red[6], S.red[7]));
+                const float uinv = pow2_above(umax), us = 1.f / uinv;   // exact powers of two
+                f16* Ud = Ug + ch * 64 * D + tid;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) Ud[i * D] = __float2half_rn(w[i] * us);
+                if (tid == 0) {
+                    SCg[ch * SC_FLOATS + SC_UINV] = uinv;
+                    SCg[ch * SC_FLOATS + SC_VMAX] = vmax;
+                }
+            }
+            tc::tc_fence_before();
+            __syncthreads();
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kPrepTmemCols);
+    return;
+abort:
+    if (tid == 0) record_timeout(status);
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kPrepTmemCols);
+}
+
+// ======================================================================================
+// chunk_carry
+// ======================================================================================
+struct CarryStage {
+    f16 A[2][128 * 64];    // [W; Q_hat] in two 64-column halves (32 KB)
+    f16 K[2][64 * 64];     // K_hat in two 64-column halves (16 KB)
+    f16 P[128 * 64];       // rows 0-63 zero, rows 64-127 P (16 KB)
+    f16 U[64 * NS];        // scaled U columns of this slice, row-major (4 KB)
+    float SC[SC_FLOATS];   // a[64], d[64], gamma_C, U scale, max |v|
+};
+struct CarrySmem {
+    CarryStage st[NSTAGE];
+    f16 H0[2][NS * 64];    // scaled fp16 state slice as K-major B operand: rows = value columns
+    f16 Dl[NS * 64];       // scaled Delta as K-major B operand (rows = value columns, K = tokens)
+    f16 Dt[NS * 64];       // scaled Delta~ = diag(exp(G_C - G)) Delta, same layout
+    float red[4];
+    uint64_t full[NSTAGE], empty[NSTAGE], bar_a, bar_bc;
+    uint32_t tmem_base;
+    volatile int abort;
+};
+constexpr size_t kCarrySmemBytes = sizeof(CarrySmem) + 1024;
+constexpr uint32_t kCarryTmemCols = 128;
+constexpr uint32_t kStageTxBytes = 2 * 128 * 64 * 2 + 2 * 64 * 64 * 2 + 64 * 64 * 2 + 64 * NS * 2 + SC_FLOATS * 4;
+
+// store the scaled fp16 copy of state row t (value columns 0..NS-1 of the slice) into
+// the K-major B operand: element (row j, column t)
+__device__ __forceinline__ void store_state_operand(f16* H0, int t, const float* h, float sc) {
+    uint8_t* base = reinterpret_cast<uint8_t*>(H0) + (t >> 6) * (NS * 128);
+    const int c = t & 63;
+#pragma unroll
+    for (int j = 0; j < NS; ++j)
+        *reinterpret_cast<f16*>(base + tc::sw128_off(j, c)) = __float2half_rn(h[j] * sc);
+}
+
+__global__ void __launch_bounds__(160, 1)
+chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qk,
+                   const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_u,
+                   const float* __restrict__ SCg, const int32_t* __restrict__ cu,
+                   const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HK, int HV,
+                   const float* __restrict__ h0, float* __restrict__ hT, bf16* __restrict__ o,
+                   int32_t* __restrict__ status) {
+    extern __shared__ uint8_t smem_raw[];
+    CarrySmem& S = *reinterpret_cast<CarrySmem*>(align1024(smem_raw));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int nslices = D / NS;
+    int idx = blockIdx.x;
+    const int vs = idx % nslices; idx /= nslices;
+    const int h = idx % HV;       idx /= HV;
+    const int n = idx;
+    const int hk = h / (HV / HK);
+    if (*reinterpret_cast<volatile int32_t*>(status) != 0) return;
+    const int64_t bos = cu ? (int64_t)cu[n] : (int64_t)n * T;
+    const int64_t len = cu ? (int64_t)cu[n + 1] - cu[n] : T;
+    const int c0 = chunk_off[n];
+    const int nch = chunk_off[n + 1] - c0;
+
+    if (warp == 0) {
+        tc::tmem_alloc(&S.tmem_base, kCarryTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (tid == 32) {
+        for (int i = 0; i < NSTAGE; ++i) {
+            tc::mbar_init(&S.full[i], 1);
+            tc::mbar_init(&S.empty[i], 1);
+        }
+        tc::mbar_init(&S.bar_a, 1);
+        tc::mbar_init(&S.bar_bc, 1);
+        tc::fence_mbar_init();
+        S.abort = 0;
+    }
+    // zero rows 0-63 of the P operands (the producer only ever writes rows 64-127)
+    for (int e = tid; e < NSTAGE * 64 * 64 / 8; e += 160) {
+        const int st = e / (64 * 64 / 8), r = e % (64 * 64 / 8);
+        reinterpret_cast<uint4*>(S.st[st].P)[r] = make_uint4(0, 0, 0, 0);
+    }
+    tc::fence_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 4) {
+        // ---------------- producer: stream the chunks through the ring ----------------
+        if (lane == 0) {
+            for (int c = 0; c < nch; ++c) {
+                const int st = c % NSTAGE, r = c / NSTAGE;
+                if (r > 0 && !tc::mbar_wait(&S.empty[st], (r - 1) & 1)) {
+                    record_timeout(status);
+                    S.abort = 1;
+                    break;
+                }
+                if (S.abort) break;
+                CarryStage& B = S.st[st];
+                const int cid = c0 + c;
+                const int row = (cid * HV + h) * 64;
+                const int qkrow = (cid * HK + hk) * 128;
+                tc::mbar_expect_tx(&S.full[st], kStageTxBytes);
+                tc::tma_load_2d(&B.A[0][0], &tm_w, &S.full[st], 0, row);
+                tc::tma_load_2d(&B.A[1][0], &tm_w, &S.full[st], 64, row);
+                tc::tma_load_2d(&B.A[0][64 * 64], &tm_qk, &S.full[st], 0, qkrow + 64);
+                tc::tma_load_2d(&B.A[1][64 * 64], &tm_qk, &S.full[st], 64, qkrow + 64);
+                tc::tma_load_2d(&B.K[0][0], &tm_qk, &S.full[st], 0, qkrow);
+                tc::tma_load_2d(&B.K[1][0], &tm_qk, &S.full[st], 64, qkrow);
+                tc::tma_load_2d(&B.P[64 * 64], &tm_p, &S.full[st], 0, row);
+                tc::tma_load_2d(B.U, &tm_u, &S.full[st], vs * NS, row);
+                tc::bulk_load(B.SC, SCg + ((size_t)cid * HV + h) * SC_FLOATS, SC_FLOATS * 4, &S.full[st]);
+            }
+        }
+    } else {
+        // ---------------- consumers: 128 threads, thread t <-> TMEM lane t -----------------
+        const int t = tid;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t tA = tmem, tB = tmem + 32, tC = tmem + 64;
+        float Hr[NS];
+        const size_t hrow = (((size_t)n * HV + h) * D + t) * D + vs * NS;
+        float m = 0.f;
+#pragma unroll
+        for (int j = 0; j < NS; ++j) {
+            Hr[j] = h0 ? h0[hrow + j] : 0.f;
+            m = fmaxf(m, fabsf(Hr[j]));
+        }
+        // data scale: fp16 operands carry x * sc with sc = 2^-e, max(|h0|, |v|) * sc < 1
+        for (int c = t; c < nch; c += 128) m = fmaxf(m, SCg[((size_t)(c0 + c) * HV + h) * SC_FLOATS + SC_VMAX]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (lane == 0) S.red[warp] = m;
+        tc::named_bar(1, 128);
+        const float inv_sc = pow2_above(fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3])));
+        const float sc = 1.f / inv_sc;
+        store_state_operand(&S.H0[0][0], t, Hr, sc);
+        tc::fence_async_smem();
+        tc::named_bar(1, 128);
+        constexpr uint32_t idA = tc::idesc_f16(128, NS, 0, 0);
+        constexpr uint32_t idB = tc::idesc_f16(128, NS, 1, 0);
+        const uint32_t h0b = tc::smem_u32(&S.H0[0][0]);
+        const uint32_t dlb = tc::smem_u32(S.Dl), dtb = tc::smem_u32(S.Dt);
+        bool failed = false;
+        for (int c = 0; c < nch; ++c) {
+            const int st = c % NSTAGE, r = c / NSTAGE;
+            CarryStage& B = S.st[st];
+            const int64_t tok = bos + (int64_t)C * c;
+            const int64_t rem = len - (int64_t)C * c;
+            const int cn = (int)(rem < C ? rem : C);
+            bool ok = tc::mbar_wait(&S.full[st], r & 1);
+            if (bar_any(1, 128, !ok)) { failed = true; break; }
+            // ---- D_a = [W; Q] H0 --------------------------------------------------------
+            if (t == 0) {
+                tc::tc_fence_after();
+                const uint32_t ab = tc::smem_u32(&B.A[0][0]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t koff = (kk & 3) * 32;
+                    tc::mma_bf16(tA, tc::desc_sw128(ab + (kk >> 2) * 16384 + koff, 16, 1024),
+                                 tc::desc_sw128(h0b + (kk >> 2) * (NS * 128) + koff, 16, 1024), idA, kk > 0);
+                }
+                tc::mma_commit(&S.bar_a);
+            }
+            ok = tc::mbar_wait(&S.bar_a, c & 1);
+            tc::tc_fence_after();
+            float x[NS];
+            tc::tmem_ld32(tA + lane_base, x);
+            tc::tmem_wait_ld();
+            const float gC = B.SC[SC_GC];
+            float op[NS];
+            if (t < 64) {   // Delta_i = U_i - (W H0)_i ; Delta~_i = d_i Delta_i   (stored scaled)
+                const float di = B.SC[64 + t], uinv = B.SC[SC_UINV];
+                const f16* urow = B.U + t * NS;
+                uint8_t* dl = reinterpret_cast<uint8_t*>(S.Dl);
+                uint8_t* dt = reinterpret_cast<uint8_t*>(S.Dt);
+#pragma unroll
+                for (int j = 0; j < NS; ++j) {
+                    const float dv = __half2float(urow[j]) * uinv - x[j] * inv_sc;
+                    const uint32_t off = tc::sw128_off(j, t);
+                    *reinterpret_cast<f16*>(dl + off) = __float2half_rn(dv * sc);
+                    *reinterpret_cast<f16*>(dt + off) = __float2half_rn(di * dv * sc);
+                }
+            } else {        // the inter-chunk part of the output rows
+                const float ai = B.SC[t - 64] * inv_sc;
+#pragma unroll
+                for (int j = 0; j < NS; ++j) op[j] = ai * x[j];
+            }
+            tc::tc_fence_before();
+            tc::fence_async_smem();
+            if (bar_any(1, 128, !ok)) { failed = true; break; }
+            // ---- D_b = K^T Delta~ (state update), D_c = [0; P] Delta (output) ------------
+            if (t == 0) {
+                tc::tc_fence_after();
+                const uint32_t kb = tc::smem_u32(&B.K[0][0]);
+                const uint32_t pb = tc::smem_u32(B.P);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tB, tc::desc_sw128(kb + kk * 2048, 8192, 1024),
+                                 tc::desc_sw128(dtb + kk * 32, 16, 1024), idB, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tC, tc::desc_sw128(pb + kk * 32, 16, 1024),
+                                 tc::desc_sw128(dlb + kk * 32, 16, 1024), idA, kk > 0);
+                tc::mma_commit(&S.bar_bc);
+                tc::mma_commit(&S.empty[st]);   // the stage's operands are consumed
+            }
+            ok = tc::mbar_wait(&S.bar_bc, c & 1);
+            tc::tc_fence_after();
+            float y[NS];
+            tc::tmem_ld32(tB + lane_base, y);
+            if (warp >= 2) tc::tmem_ld32(tC + lane_base, x);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < NS; ++j) Hr[j] = fmaf(gC, Hr[j], y[j] * inv_sc);
+            store_state_operand(&S.H0[0][0], t, Hr, sc);
+            if (t >= 64 && t - 64 < cn) {
+                __align__(16) bf16 ob[NS];
+#pragma unroll
+                for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(x[j], inv_sc, op[j]));
+                uint4* dst = reinterpret_cast<uint4*>(o + ((tok + t - 64) * HV + h) * D + vs * NS);
+#pragma unroll
+                for (int q = 0; q < NS / 8; ++q) dst[q] = reinterpret_cast<const uint4*>(ob)[q];
+            }
+            tc::tc_fence_before();
+            tc::fence_async_smem();
+            if (bar_any(1, 128, !ok)) { failed = true; break; }
+        }
+        if (failed) {
+            if (t == 0) record_timeout(status);
+            S.abort = 1;
+        } else if (hT) {
+#pragma unroll
+            for (int j = 0; j < NS; ++j) hT[hrow + j] = Hr[j];
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (S.abort && tid == 0) {
+        // let copies already issued land before the shared memory is released
+        for (int i = 0; i < NSTAGE; ++i) (void)tc::mbar_wait(&S.full[i], 0, 50000000ull);
+    }
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kCarryTmemCols);
+}
+
+// ======================================================================================
+// host side
+// ======================================================================================
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct TcLayout {
+    int64_t max_chunks;
+    size_t off_chunk, off_w, off_u, off_p, off_qk, off_sc, total;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Upper bound on the chunk count of any split of n_tokens into n_seqs sequences (each
+// sequence adds at most one partial chunk); used for dense and packed layouts alike.
+TcLayout tc_layout(int64_t n_tokens, int n_seqs, int HK, int HV) {
+    TcLayout L;
+    L.max_chunks = (n_tokens + C - 1) / C + n_seqs;
+    const size_t rows = (size_t)L.max_chunks * HV * 64;
+    L.off_chunk = kStatusBytes;
+    L.off_w = round_up(L.off_chunk + (size_t)(n_seqs + 1) * 4, 1024);
+    L.off_u = round_up(L.off_w + rows * D * 2, 1024);
+    L.off_p = round_up(L.off_u + rows * D * 2, 1024);
+    L.off_qk = round_up(L.off_p + rows * 64 * 2, 1024);
+    L.off_sc = round_up(L.off_qk + (size_t)L.max_chunks * HK * 128 * D * 2, 1024);
+    L.total = round_up(L.off_sc + (size_t)L.max_chunks * HV * SC_FLOATS * 4, 1024);
+    return L;
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int Dk, int Dv, int HK, int HV, int BT) {
+    return Dk == D && Dv == D && BT == C && (HV / HK == 1 || HV / HK == 2);
+}
+
+size_t prefill_tc_workspace_bytes(int64_t n_tokens, int n_seqs, int HK, int HV) {
+    return tc_layout(n_tokens, n_seqs, HK, HV).total;
+}
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_t s) {
+    const bool packed = a.cu != nullptr;
+    const int64_t n_tokens = packed ? a.T : (int64_t)a.n_seqs * a.T;
+    const TcLayout L = tc_layout(n_tokens, a.n_seqs, a.HK, a.HV);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* chunk_off = reinterpret_cast<int32_t*>(ws + L.off_chunk);
+    f16* W = reinterpret_cast<f16*>(ws + L.off_w);
+    f16* U = reinterpret_cast<f16*>(ws + L.off_u);
+    f16* P = reinterpret_cast<f16*>(ws + L.off_p);
+    f16* QK = reinterpret_cast<f16*>(ws + L.off_qk);
+    float* SC = reinterpret_cast<float*>(ws + L.off_sc);
+
+    chunk_table_kernel<<<1, 1024, 0, s>>>(a.cu, a.n_seqs, a.T, chunk_off, a.status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch();
+    if (n_tokens == 0 && a.hT == nullptr) return cudaSuccess;
+
+    // tensor maps: bf16 inputs for the chunk-local stage, fp16 intermediates for the carry
+    CUtensorMap tq, tk, tv, tw, tu, tp, tqk;
+    const cuuint64_t tok = (cuuint64_t)(n_tokens > 0 ? n_tokens : 1);
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.HK, tok};
+        cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.HK * D * 2};
+        cuuint32_t box[3] = {64, 1, 64};
+        const void* qb = a.q ? a.q : workspace;
+        const void* kb = a.k ? a.k : workspace;
+        if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qb, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kb, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.HV, tok};
+        cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.HV * D * 2};
+        cuuint32_t box[3] = {64, 1, 64};
+        const void* vb = a.v ? a.v : workspace;
+        if (!make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, vb, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+    const cuuint64_t mc = (cuuint64_t)(L.max_chunks > 0 ? L.max_chunks : 1);
+    const cuuint64_t rows = mc * a.HV * 64;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)D, rows};
+        cuuint64_t str[1] = {(cuuint64_t)D * 2};
+        cuuint32_t box[2] = {64, 64};
+        if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, W, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        cuuint32_t boxu[2] = {NS, 64};
+        if (!make_map(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, U, 2, dims, str, boxu, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[2] = {64, rows};
+        cuuint64_t str[1] = {64 * 2};
+        cuuint32_t box[2] = {64, 64};
+        if (!make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, P, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)D, mc * a.HK * 128};
+        cuuint64_t str[1] = {(cuuint64_t)D * 2};
+        cuuint32_t box[2] = {64, 64};
+        if (!make_map(&tqk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, QK, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+
+    const int G = a.HV / a.HK;
+    if (n_tokens > 0 && L.max_chunks > 0) {
+        dim3 grid((unsigned)L.max_chunks, (unsigned)a.HK);
+        if (G == 1) {
+            e = cudaFuncSetAttribute(chunk_prep_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kPrepSmemBytes);
+            if (e != cudaSuccess) return e;
+            chunk_prep_kernel<1><<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T,
+                                                                 a.n_seqs, a.HV, a.scale, a.l2norm, a.HK, W, U, P,
+                                                                 QK, SC, a.status);
+        } else {
+            e = cudaFuncSetAttribute(chunk_prep_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kPrepSmemBytes);
+            if (e != cudaSuccess) return e;
+            chunk_prep_kernel<2><<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T,
+                                                                 a.n_seqs, a.HV, a.scale, a.l2norm, a.HK, W, U, P,
+                                                                 QK, SC, a.status);
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        count_launch();
+    }
+    e = cudaFuncSetAttribute(chunk_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCarrySmemBytes);
+    if (e != cudaSuccess) return e;
+    const unsigned blocks = (unsigned)a.n_seqs * (unsigned)a.HV * (unsigned)(D / NS);
+    chunk_carry_kernel<<<blocks, 160, kCarrySmemBytes, s>>>(tw, tqk, tp, tu, SC, a.cu, chunk_off, a.T, a.n_seqs,
+                                                          a.HK, a.HV, a.h0, a.hT, (bf16*)a.o, a.status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch();
+    return cudaSuccess;
+}
+
+}  // namespace gdn

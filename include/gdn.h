@@ -64,6 +64,7 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 /* Device-side error codes written into the prefill workspace's status word. */
 #define GDN_DEVERR_NONE 0
 #define GDN_DEVERR_CU_SEQLENS 1   /* cu_seqlens[0] != 0, decreasing, or last != T */
+#define GDN_DEVERR_TIMEOUT 2      /* a bounded wait inside a kernel expired; outputs invalid */
 
 /* Human-readable name of a gdn_status value (static storage, never NULL). */
 GDN_API const char* gdn_status_string(int status);
@@ -127,6 +128,8 @@ GDN_API size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seq
  *                 not be shared by calls that may run concurrently.
  *   BT            chunk length: 64 (GDN_BF16) or 16, 32, 64 (GDN_F32).  BT only
  *                 changes rounding, never the result's definition.
+ *                 GDN_BF16 with Dk = Dv = 128 and HV / HK in {1, 2} runs on the tensor
+ *                 cores (tcgen05); other GDN_BF16 shapes and GDN_F32 run on CUDA cores.
  *   scale         multiplies o (1.0 = the plain rule).
  *   qk_l2norm     nonzero: q and k rows are replaced by x / sqrt(sum x^2 + 1e-6)
  *                 before use (per token and q/k head).

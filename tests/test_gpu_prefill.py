@@ -152,7 +152,8 @@ def test_bad_cu_seqlens_reported_and_nothing_written():
         assert G.gdn_chunk_prefill_status(ws) == 1
         assert torch.all(o == 5.0) and torch.all(hT == 9.0)
     cu = torch.tensor([0, 40, 96], dtype=torch.int32, device="cuda")
-    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(G.prefill_workspace_bytes(96, 2, 1, 2, 128, 128, 64, 1), dtype=torch.uint8,
+                     device="cuda")
     G.gdn_chunk_prefill(q, k, v, g, g, cu_seqlens=cu, workspace=ws)
     assert G.gdn_chunk_prefill_status(ws) == 0
 
