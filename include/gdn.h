@@ -158,6 +158,40 @@ GDN_API gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v
 GDN_API gdn_status gdn_chunk_prefill_status(const void* workspace, void* stream, int32_t* device_error);
 
 /*
+ * gdn_chunk_prefill_static_ws -- gdn_chunk_prefill without a caller-provided workspace.
+ * The pages describe no such call: it exists for callers whose host code may not
+ * allocate device memory (a serving loop under a no-allocation rule, where an
+ * allocation can synchronise the device; code called back from a framework that owns
+ * the device memory and offers no allocator).  Arguments, layouts and results are those
+ * of gdn_chunk_prefill minus workspace / workspace_bytes; nothing is allocated or freed.
+ *
+ * The scratch is one file-scope device array of GDN_STATIC_SCRATCH_BYTES inside the
+ * library, present on every GPU that loads the library until the process exits.
+ *   - Sizes whose gdn_chunk_prefill_workspace_bytes(...) exceeds GDN_STATIC_SCRATCH_BYTES
+ *     are rejected with GDN_ERR_WORKSPACE before anything is launched (for bf16, 128-dim
+ *     heads that is about 2K tokens at 32 value heads).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ *     capture on that device.
+ *   - Every call on a device shares the one array, and it keeps the previous call's
+ *     contents; each call rewrites all of it that it reads, so nothing needs clearing.
+ *     Calls whose executions overlap on the GPU (other streams, other host threads)
+ *     race on the array and give wrong results: serialise them.
+ *   - The device status word lives in the array, so a bad cu_seqlens table (outputs left
+ *     unwritten) cannot be read back through this call; validate the table beforehand.
+ * Errors: those of gdn_chunk_prefill, GDN_ERR_WORKSPACE for sizes over the cap, and
+ * GDN_ERR_CUDA if the array's address cannot be obtained.
+ */
+#define GDN_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+GDN_API gdn_status gdn_chunk_prefill_static_ws(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                             const float* g, const float* beta,
+                             const float* initial_state, const int32_t* cu_seqlens,
+                             int32_t B, int64_t T, int32_t n_seqs,
+                             int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                             int32_t BT, float scale, int32_t qk_l2norm,
+                             void* o, float* final_state, void* stream);
+
+/*
  * gdn_decode_step -- one token per sequence, state updated in place (the
  * incremental update of the "QWEN3.5" Q&A page, question 2a: decay the whole
  * state by alpha, then clear and write along the current key with strength beta).
