@@ -21,7 +21,6 @@ from __future__ import annotations
 import argparse
 import json
 import os
-import shutil
 import statistics
 import subprocess
 import sys
@@ -67,57 +66,80 @@ def decode_bytes_per_step(B, HK, HV, Dk, Dv, io_bytes=2):
 
 # ---------------------------------------------------------------------------
 class Clocks:
-    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event (throttle) reasons sampled every 2 ms through NVML
+    from a background thread; only samples inside the timed regions (host wall-clock
+    windows added with ``window``) are summarised.  Reads settings only."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80))
 
     def __init__(self, device_index: int):
         self.dev = device_index
-        self.proc = None
-        self.path = None
+        self.windows = []
+        self.samples = []
+        self.thread = None
+        self.stop_flag = False
+        self.err = None
+
+    def window(self, t0: float, t1: float):
+        self.windows.append((t0, t1))
+
+    def _handle(self, nv):
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
-        exe = shutil.which("nvidia-smi")
-        if not exe:
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+        except Exception as e:  # pragma: no cover
+            self.err = f"NVML unavailable: {e}"
             return
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        self.proc = subprocess.Popen([exe, f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                      "-i", str(self.dev), "-lms", "100"],
-                                     stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+
+        def loop():
+            while not self.stop_flag:
+                try:
+                    self.samples.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                         int(get_reasons(h)), nv.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception as e:  # pragma: no cover
+                    self.err = str(e)
+                    return
+                time.sleep(0.002)
+
+        self.nv = nv
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
-                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        load = [r for r in rows if r["power"] > 0.5 * max(x["power"] for x in rows)] or rows
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "not sampled"]}
+        self.stop_flag = True
+        self.thread.join(2)
+        inside = [x for x in self.samples if any(a <= x[0] <= b for a, b in self.windows)]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.smax, "samples": 0,
+                    "reasons": ["no samples inside the timed regions"]}
         reasons = set()
-        for r in rows:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
-                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
-                if r[key].lower().startswith("active"):
+        for _, _, bits, _ in inside:
+            for name, attr, default in self.REASONS:
+                if bits & getattr(self.nv, attr, default):
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": rows[0]["smax"],
-                "reasons": sorted(reasons), "samples": len(rows),
-                "power_w_max": max(r["power"] for r in rows)}
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": self.smax,
+                "reasons": sorted(reasons), "samples": len(inside),
+                "power_w_max": max(x[3] for x in inside), "sampled": "NVML every 2 ms, timed regions only"}
 
 
 # ---------------------------------------------------------------------------
@@ -228,11 +250,12 @@ def run_gdn(args, rank, world, dist):
             "dtype": "bf16", "data": "synthetic"}
     if do_prefill:
         clocks.start()
-        line.update(bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_over_ranks))
+        line.update(bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_over_ranks,
+                                  clocks))
     if do_decode:
         if not do_prefill:
             clocks.start()
-        line["decode"] = bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks)
+        line["decode"] = bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, clocks)
     line["clocks"] = clocks.stop()
     if do_prefill and rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, T_s, t, th = cpu_oracle_sample(args.cpu_seconds, T)
@@ -250,7 +273,7 @@ def _traffic():
     return {}
 
 
-def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_over_ranks):
+def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_over_ranks, clocks):
     import numpy as np
     import statistics
     import torch
@@ -283,11 +306,13 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     n0 = G.kernel_launches()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
     t0.record()
     for i in range(args.steps):
         prefill_step(kev[i])
     t1.record()
     barrier()
+    clocks.window(w0, time.time())
     launches = G.kernel_launches() - n0
     ms_local = t0.elapsed_time(t1) / args.steps
     kernel_ms_local = statistics.mean(e0.elapsed_time(e1) for e0, e1 in kev)
@@ -348,7 +373,7 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     }
 
 
-def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks):
+def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, clocks):
     import torch
     import gated_deltanet_sequence_delta_b200 as G
     from gated_deltanet_sequence_delta_b200 import inputs as I
@@ -375,22 +400,26 @@ def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks):
     d0 = torch.cuda.Event(enable_timing=True)
     d1 = torch.cuda.Event(enable_timing=True)
     nd0 = G.kernel_launches()
+    w0 = time.time()
     d0.record()
     for i in range(n_dec):
         decode_step(i)
     d1.record()
     barrier()
+    clocks.window(w0, time.time())
     dec_launches = G.kernel_launches() - nd0
     dec_ms = max_over_ranks(d0.elapsed_time(d1) / n_dec)
     # the decode kernel alone, same inputs, back to back
     dq, dk, dv, _, _ = ring[0]
     k0 = torch.cuda.Event(enable_timing=True)
     k1 = torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
     k0.record()
     for i in range(n_dec):
         G.gdn_decode_step(dq, dk, dv, dg, dbeta, state, o=do)
     k1.record()
     barrier()
+    clocks.window(w0, time.time())
     dec_kernel_ms = max_over_ranks(k0.elapsed_time(k1) / n_dec)
     dbytes = decode_bytes_per_step(ds.B, ds.HK, ds.HV, ds.Dk, ds.Dv)
     dgbs = dbytes / (dec_kernel_ms * 1e-3) / 1e9
