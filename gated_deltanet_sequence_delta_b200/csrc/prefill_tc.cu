@@ -152,121 +152,107 @@ __global__ void __launch_bounds__(1024) chunk_table_kernel(const int32_t* __rest
 }
 
 // ======================================================================================
-// T = (I + L)^-1 for a 64 x 64 strictly lower L (fp32, row stride 65), 128 threads.
-// Writes the lower triangle of T including its unit diagonal; entries above the diagonal
-// are left untouched.  Blocks of 16: T_ii = (I + L_ii)^-1 by column substitution, then
-// T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj by increasing i - j.
+// In-place T = (I + L)^-1 for a 64 x 64 strictly lower L held in M (fp32, row stride 65),
+// 128 threads.  On return the strictly lower triangle of M holds T (its unit diagonal is
+// implied); entries on and above the diagonal are untouched.  Blocks of 16:
+//  * diagonal blocks T_bb = (I + L_bb)^-1 by right-looking column substitution: every
+//    finished x_j updates all later rows at once, so the dependent chain is one FMA per row;
+//  * block rows I = 1, 2, 3: T_Ij = -T_II sum_{k=j}^{I-1} L_Ik T_kj for all j < I at once.
+//    Row block I of L is read only while row block I of T is formed, so T overwrites it.
 // ======================================================================================
-__device__ __forceinline__ void tinv64(const float (*L)[65], float (*Tm)[65], float (*X)[16][17], int tid) {
+template <int I>
+__device__ __forceinline__ void tinv_row_block(float (*M)[65], float (*X)[16][17], int tid) {
+    const int c = tid & 15, r0 = tid >> 4;   // this thread: rows r0 and r0 + 8, column c
+    float acc[I][2];
+#pragma unroll
+    for (int j = 0; j < I; ++j) acc[j][0] = acc[j][1] = 0.f;
+#pragma unroll
+    for (int j = 0; j < I; ++j) {
+#pragma unroll
+        for (int k = j; k < I; ++k) {
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) {
+                float t;
+                if (k == j) t = kk == c ? 1.f : (kk > c ? M[16 * j + kk][16 * j + c] : 0.f);
+                else t = M[16 * k + kk][16 * j + c];
+                acc[j][0] = fmaf(M[16 * I + r0][16 * k + kk], t, acc[j][0]);
+                acc[j][1] = fmaf(M[16 * I + r0 + 8][16 * k + kk], t, acc[j][1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < I; ++j) {
+        X[j][r0][c] = acc[j][0];
+        X[j][r0 + 8][c] = acc[j][1];
+    }
+    __syncthreads();   // every read of row block I of L is done before it is overwritten
+#pragma unroll
+    for (int j = 0; j < I; ++j) {
+        float a0 = X[j][r0][c], a1 = X[j][r0 + 8][c];
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            const float xk = X[j][kk][c];
+            if (kk < r0) a0 = fmaf(M[16 * I + r0][16 * I + kk], xk, a0);
+            if (kk < r0 + 8) a1 = fmaf(M[16 * I + r0 + 8][16 * I + kk], xk, a1);
+        }
+        acc[j][0] = -a0;
+        acc[j][1] = -a1;
+    }
+#pragma unroll
+    for (int j = 0; j < I; ++j) {
+        M[16 * I + r0][16 * j + c] = acc[j][0];
+        M[16 * I + r0 + 8][16 * j + c] = acc[j][1];
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void tinv64_inplace(float (*M)[65], float (*X)[16][17], int tid) {
+    float col[16];
+    const int b = tid >> 4, c = tid & 15, o = 16 * b;
     if (tid < 64) {
-        const int b = tid >> 4, c = tid & 15, o = 16 * b;
-        float x[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float acc = (i == c) ? 1.f : 0.f;
+        for (int i = 0; i < 16; ++i) col[i] = (i == c) ? 1.f : 0.f;
 #pragma unroll
-            for (int j = 0; j < i; ++j) acc = fmaf(-L[o + i][o + j], x[j], acc);
-            x[i] = acc;
+        for (int j = 0; j < 15; ++j) {
+            const float xj = col[j];
+#pragma unroll
+            for (int i = j + 1; i < 16; ++i) col[i] = fmaf(-M[o + i][o + j], xj, col[i]);
         }
+    }
+    __syncthreads();   // all reads of the diagonal blocks of L precede their overwrite
+    if (tid < 64) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (i >= c) Tm[o + i][o + c] = x[i];
+        for (int i = 1; i < 16; ++i)
+            if (i > c) M[o + i][o + c] = col[i];
     }
     __syncthreads();
-    // first sub-diagonal blocks (b+1, b), b = 0, 1, 2
-    for (int e = tid; e < 3 * 256; e += 128) {
-        const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
-        const int oi = 16 * (b + 1), oj = 16 * b;
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-            if (k >= c) acc = fmaf(L[oi + r][oj + k], Tm[oj + k][oj + c], acc);
-        X[b][r][c] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < 3 * 256; e += 128) {
-        const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
-        const int oi = 16 * (b + 1), oj = 16 * b;
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-            if (k <= r) acc = fmaf(Tm[oi + r][oi + k], X[b][k][c], acc);
-        Tm[oi + r][oj + c] = -acc;
-    }
-    __syncthreads();
-    // second sub-diagonal blocks (2, 0) and (3, 1)
-    for (int e = tid; e < 2 * 256; e += 128) {
-        const int p = e >> 8, r = (e >> 4) & 15, c = e & 15;
-        const int oi = 16 * (p + 2), oj = 16 * p, om = 16 * (p + 1);
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            if (k >= c) acc = fmaf(L[oi + r][oj + k], Tm[oj + k][oj + c], acc);
-            acc = fmaf(L[oi + r][om + k], Tm[om + k][oj + c], acc);
-        }
-        X[p][r][c] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < 2 * 256; e += 128) {
-        const int p = e >> 8, r = (e >> 4) & 15, c = e & 15;
-        const int oi = 16 * (p + 2), oj = 16 * p;
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-            if (k <= r) acc = fmaf(Tm[oi + r][oi + k], X[p][k][c], acc);
-        Tm[oi + r][oj + c] = -acc;
-    }
-    __syncthreads();
-    // third sub-diagonal block (3, 0)
-    for (int e = tid; e < 256; e += 128) {
-        const int r = e >> 4, c = e & 15;
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            if (k >= c) acc = fmaf(L[48 + r][k], Tm[k][c], acc);
-            acc = fmaf(L[48 + r][16 + k], Tm[16 + k][c], acc);
-            acc = fmaf(L[48 + r][32 + k], Tm[32 + k][c], acc);
-        }
-        X[0][r][c] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < 256; e += 128) {
-        const int r = e >> 4, c = e & 15;
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-            if (k <= r) acc = fmaf(Tm[48 + r][48 + k], X[0][k][c], acc);
-        Tm[48 + r][c] = -acc;
-    }
-    __syncthreads();
+    tinv_row_block<1>(M, X, tid);
+    tinv_row_block<2>(M, X, tid);
+    tinv_row_block<3>(M, X, tid);
 }
 
 // ======================================================================================
 // chunk_prep
 // ======================================================================================
 struct PrepSmem {
-    bf16 KQ[2][128 * 64];   // two 64-column halves of [K; Q] (rows 0-63 K, 64-127 Q), 16 KB each
-    bf16 V[2][64 * 64];     // two 64-column halves of V, 8 KB each
-    bf16 AW[64 * 64];       // hi part of T diag(b gamma rk), K-major B operand (rows i, K = j)
-    bf16 AU[64 * 64];       // hi part of T diag(b)
-    union {                 // L is dead once T is formed; its space then holds the lo parts
-        float L[64][65];
-        struct {
-            bf16 AWlo[64 * 64];
-            bf16 AUlo[64 * 64];
-        } lo;
-    } u;
-    float Tm[64][65];
+    // [K; Q] in two 64-column halves (rows 0-63 K, 64-127 Q), 16 KB each.  Rows 0-63 are
+    // rewritten in place as fp16 K_hat; rows 64-127 are reused for V (bf16 from TMA, then
+    // fp16 V * sv in place) once Q_hat has been written out.
+    uint16_t KQ[2][128 * 64];
+    f16 AW[64 * 64];        // T diag(b gamma) as K-major B operand (rows i, K = j); later
+    f16 AU[64 * 64];        //   AW..AU stage the fp16 W tile on its way to global memory
+    float M[64][65];        // L, then T in place; later stages the U tile
     float X[3][16][17];
     float rk[64], rq[64], G[64], bt[64], bgr[64], red[8];
+    float ga[2][64], ba[2][64];   // prefetched g, beta of the (up to two) value heads
     uint64_t bar_load, bar_v, bar_mma;
     uint32_t tmem_base;
 };
 constexpr size_t kPrepSmemBytes = sizeof(PrepSmem) + 1024;
-constexpr uint32_t kPrepTmemCols = 256;
+constexpr uint32_t kPrepTmemCols = 128;
 
 template <int G>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(128, 3)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
                   const float* __restrict__ beta, const int32_t* __restrict__ cu,
@@ -297,26 +283,32 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc::tc_fence_after();
     const uint32_t tmem = S.tmem_base;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t tD1 = tmem, tDW = tmem + 64, tDU = tmem + 128;
+    const uint32_t tD1 = tmem, tDU = tmem, tDW = tmem + 64;   // D_U reuses D1's columns
     const int si = (int)s;
+    uint8_t* kq = reinterpret_cast<uint8_t*>(&S.KQ[0][0]);
 
     if (tid == 0) {
         tc::mbar_expect_tx(&S.bar_load, 4 * 64 * 64 * 2);
-        tc::tma_load_3d(&S.KQ[0][0], &tm_k, &S.bar_load, 0, hk, si);
-        tc::tma_load_3d(&S.KQ[1][0], &tm_k, &S.bar_load, 64, hk, si);
-        tc::tma_load_3d(&S.KQ[0][64 * 64], &tm_q, &S.bar_load, 0, hk, si);
-        tc::tma_load_3d(&S.KQ[1][64 * 64], &tm_q, &S.bar_load, 64, hk, si);
-        tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
-        tc::tma_load_3d(&S.V[0][0], &tm_v, &S.bar_v, 0, hk * G, si);
-        tc::tma_load_3d(&S.V[1][0], &tm_v, &S.bar_v, 64, hk * G, si);
+        tc::tma_load_3d(kq, &tm_k, &S.bar_load, 0, hk, si);
+        tc::tma_load_3d(kq + 16384, &tm_k, &S.bar_load, 64, hk, si);
+        tc::tma_load_3d(kq + 8192, &tm_q, &S.bar_load, 0, hk, si);
+        tc::tma_load_3d(kq + 16384 + 8192, &tm_q, &S.bar_load, 64, hk, si);
+    }
+    if (tid < 64) {   // gates of the group's value heads, prefetched under the TMA latency
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) {
+            const int h = hk * G + gi;
+            S.ga[gi][tid] = tid < cn ? g[(s + tid) * HV + h] : 0.f;
+            S.ba[gi][tid] = tid < cn ? beta[(s + tid) * HV + h] : 0.f;
+        }
     }
     bool ok = tc::mbar_wait(&S.bar_load, 0);
     if (__syncthreads_or(!ok)) goto abort;
 
-    // ---- Gram tiles: D1[0:64] = K K^T, D1[64:128] = Q K^T (M=128, N=64, K=Dk) ---------
+    // ---- Gram tiles: D1[0:64] = K K^T, D1[64:128] = Q K^T (bf16, M=128, N=64, K=Dk) ----
     if (tid == 0) {
         tc::tc_fence_after();
-        const uint32_t base = tc::smem_u32(&S.KQ[0][0]);
+        const uint32_t base = tc::smem_u32(kq);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint64_t d = tc::desc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
@@ -324,11 +316,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         tc::mma_commit(&S.bar_mma);
     }
-    if (tid >= 64) {   // inverse norms of q rows, from the raw tile (order inside a row is irrelevant)
+    if (tid >= 64) {   // inverse norms of q rows (order inside a row is irrelevant)
         float ss = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-            const uint4* row = reinterpret_cast<const uint4*>(&S.KQ[half][tid * 64]);
+            const uint4* row = reinterpret_cast<const uint4*>(kq + half * 16384 + tid * 128);
 #pragma unroll
             for (int c16 = 0; c16 < 8; ++c16) {
                 const uint4 u = row[c16];
@@ -360,45 +352,55 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         __syncthreads();
         const float rki = tid < 64 ? S.rk[tid] : 0.f;
         const float rqi = tid >= 64 ? S.rq[tid - 64] : 0.f;
-        {   // normalised fp16 copies of this row of K (tid < 64) or Q, in natural column order
-            const float rr = tid < 64 ? rki : rqi;
+        {   // K_hat (tid < 64) / Q_hat row: fp16 in place (K_hat feeds the W MMA) and out to
+            // global in natural column order; rows past the chunk are zeroed
+            const float rr = tid < cn || (tid >= 64 && tid - 64 < cn) ? (tid < 64 ? rki : rqi) : 0.f;
             uint4* dst = reinterpret_cast<uint4*>(QKg + (((size_t)chunk * HK + hk) * 128 + tid) * D);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                const uint4* row = reinterpret_cast<const uint4*>(&S.KQ[half][tid * 64]);
+                uint4* row = reinterpret_cast<uint4*>(kq + half * 16384 + tid * 128);
 #pragma unroll
                 for (int c16 = 0; c16 < 8; ++c16) {
-                    const uint4 u = row[c16 ^ (tid & 7)];   // logical chunk c16 sits at c16 ^ (row % 8)
+                    const int pc = c16 ^ (tid & 7);   // logical chunk c16 sits at c16 ^ (row % 8)
+                    const uint4 u = row[pc];
                     const bf16* e = reinterpret_cast<const bf16*>(&u);
                     __align__(16) f16 hx[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) hx[t] = __float2half_rn(__bfloat162float(e[t]) * rr);
-                    dst[half * 8 + c16] = *reinterpret_cast<const uint4*>(hx);
+                    const uint4 hv = *reinterpret_cast<const uint4*>(hx);
+                    row[pc] = hv;
+                    dst[half * 8 + c16] = hv;
                 }
             }
+        }
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {   // Q is consumed: its rows now receive V of the first value head
+            tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+            tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, hk * G, si);
+            tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, hk * G, si);
         }
 
         for (int gi = 0; gi < G; ++gi) {
             const int h = hk * G + gi;
             const size_t ch = (size_t)chunk * HV + h;
-            // ---- gates of this value head: running sum of g, write strengths ---------
+            // ---- running sum of the log-decays, write strengths -------------------------
             if (tid < 64) {
-                float gv = tid < cn ? g[(s + tid) * HV + h] : 0.f;
-                const float bv = tid < cn ? beta[(s + tid) * HV + h] : 0.f;
+                float gv = S.ga[gi][tid];
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, gv, o);
                     if ((tid & 31) >= o) gv += y;
                 }
                 S.G[tid] = gv;
-                S.bt[tid] = bv;
+                S.bt[tid] = S.ba[gi][tid];
             }
             __syncthreads();
             if (tid >= 32 && tid < 64) S.G[tid] += S.G[31];
             __syncthreads();
-            if (tid < 64) S.bgr[tid] = S.bt[tid] * expf(S.G[tid]) * S.rk[tid];
+            if (tid < 64) S.bgr[tid] = S.bt[tid] * expf(S.G[tid]);
             const float Gl = S.G[63];   // padding adds 0, so this is G at the last token
-            // ---- L (strictly lower) and P (lower incl. diagonal), scalars -----------------
+            // ---- L (strictly lower) into M, P (lower incl. diagonal) out, scalars ------
             if (tid < 64) {
                 const int i = tid;
                 const float Gi = S.G[i], bi = S.bt[i] * rki;
@@ -406,7 +408,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int j = 0; j < 64; ++j) {
                     float v = 0.f;
                     if (j < i && i < cn) v = bi * expf(Gi - S.G[j]) * S.rk[j] * row[j];
-                    S.u.L[i][j] = v;
+                    S.M[i][j] = v;
                 }
                 SCg[ch * SC_FLOATS + 64 + i] = i < cn ? expf(Gl - Gi) : 0.f;
             } else {
@@ -429,42 +431,36 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
             __syncthreads();
-            tinv64(S.u.L, S.Tm, S.X, tid);
-            // ---- MMA operands T diag(b gamma rk) and T diag(b) as bf16 hi + lo parts ------
+            tinv64_inplace(S.M, S.X, tid);
+            // ---- fp16 MMA operands T diag(b gamma) and T diag(b), 128B-swizzled ----------
             {
                 const int i = tid >> 1, c0 = (tid & 1) * 32;
                 uint8_t* aw = reinterpret_cast<uint8_t*>(S.AW);
                 uint8_t* au = reinterpret_cast<uint8_t*>(S.AU);
-                uint8_t* awl = reinterpret_cast<uint8_t*>(S.u.lo.AWlo);
-                uint8_t* aul = reinterpret_cast<uint8_t*>(S.u.lo.AUlo);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    __align__(16) bf16 w8[8], u8[8], wl8[8], ul8[8];
+                    __align__(16) f16 w8[8], u8[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
                         const int j = c0 + cc * 8 + t;
-                        const float tij = j < i ? S.Tm[i][j] : (j == i ? 1.f : 0.f);
-                        const float wv = tij * S.bgr[j], uv = tij * S.bt[j];
-                        w8[t] = __float2bfloat16_rn(wv);
-                        u8[t] = __float2bfloat16_rn(uv);
-                        wl8[t] = __float2bfloat16_rn(wv - __bfloat162float(w8[t]));
-                        ul8[t] = __float2bfloat16_rn(uv - __bfloat162float(u8[t]));
+                        const float tij = j < i ? S.M[i][j] : (j == i ? 1.f : 0.f);
+                        w8[t] = __float2half_rn(tij * S.bgr[j]);
+                        u8[t] = __float2half_rn(tij * S.bt[j]);
                     }
                     const uint32_t off = tc::sw128_off(i, c0 + cc * 8);
                     *reinterpret_cast<uint4*>(aw + off) = *reinterpret_cast<const uint4*>(w8);
                     *reinterpret_cast<uint4*>(au + off) = *reinterpret_cast<const uint4*>(u8);
-                    *reinterpret_cast<uint4*>(awl + off) = *reinterpret_cast<const uint4*>(wl8);
-                    *reinterpret_cast<uint4*>(aul + off) = *reinterpret_cast<const uint4*>(ul8);
                 }
             }
-            tc::fence_async_smem();
+            // ---- V tile of this head: max |v|, then fp16(v * sv) in place, rows past the
+            //      chunk zeroed -----------------------------------------------------------
             ok = tc::mbar_wait(&S.bar_v, gi & 1);
             if (__syncthreads_or(!ok)) goto abort;
-            float vmax = 0.f;   // max |v| over the tile (rows past the chunk are masked out)
             {
-                const int r = tid >> 1;
+                const int r = tid >> 1, half = tid & 1;
+                uint4* vr = reinterpret_cast<uint4*>(kq + half * 16384 + 8192 + r * 128);
+                float vmax = 0.f;
                 if (r < cn) {
-                    const uint4* vr = reinterpret_cast<const uint4*>(&S.V[tid & 1][r * 64]);
 #pragma unroll
                     for (int c16 = 0; c16 < 8; ++c16) {
                         const uint4 u = vr[c16];
@@ -473,78 +469,82 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         for (int t = 0; t < 8; ++t) vmax = fmaxf(vmax, fabsf(__bfloat162float(e[t])));
                     }
                 }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+                if ((tid & 31) == 0) S.red[warp] = vmax;
+                __syncthreads();
+                vmax = fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3]));
+                const float uinv = pow2_above(vmax), sv = r < cn ? 1.f / uinv : 0.f;
+#pragma unroll
+                for (int c16 = 0; c16 < 8; ++c16) {
+                    const uint4 u = vr[c16];
+                    const bf16* e = reinterpret_cast<const bf16*>(&u);
+                    __align__(16) f16 hx[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) hx[t] = __float2half_rn(__bfloat162float(e[t]) * sv);
+                    vr[c16] = *reinterpret_cast<const uint4*>(hx);
+                }
+                if (tid == 0) {
+                    SCg[ch * SC_FLOATS + SC_UINV] = uinv;
+                    SCg[ch * SC_FLOATS + SC_VMAX] = vmax;
+                }
             }
-            // ---- W^T = K^T AW^T and U^T = V^T AU^T (M=128, N=64, K=64 tokens) -----------
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            __syncthreads();
+            // ---- W^T = K_hat^T AW^T and (V sv)^T AU^T (fp16, M=128, N=64, K=64 tokens) ----
             if (tid == 0) {
                 tc::tc_fence_after();
-                const uint32_t kb = tc::smem_u32(&S.KQ[0][0]);
-                const uint32_t vb = tc::smem_u32(&S.V[0][0]);
+                const uint32_t kb = tc::smem_u32(kq), vb = kb + 8192;
                 const uint32_t awb = tc::smem_u32(S.AW), aub = tc::smem_u32(S.AU);
-                const uint32_t awl = tc::smem_u32(S.u.lo.AWlo), aul = tc::smem_u32(S.u.lo.AUlo);
-                constexpr uint32_t idx = tc::idesc_bf16(128, 64, 1, 0);
+                constexpr uint32_t idx = tc::idesc_f16(128, 64, 1, 0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tDW, tc::desc_sw128(kb + kk * 2048, 16384, 1024),
                                  tc::desc_sw128(awb + kk * 32, 16, 1024), idx, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tDW, tc::desc_sw128(kb + kk * 2048, 16384, 1024),
-                                 tc::desc_sw128(awl + kk * 32, 16, 1024), idx, 1);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tDU, tc::desc_sw128(vb + kk * 2048, 8192, 1024),
+                    tc::mma_bf16(tDU, tc::desc_sw128(vb + kk * 2048, 16384, 1024),
                                  tc::desc_sw128(aub + kk * 32, 16, 1024), idx, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tDU, tc::desc_sw128(vb + kk * 2048, 8192, 1024),
-                                 tc::desc_sw128(aul + kk * 32, 16, 1024), idx, 1);
                 tc::mma_commit(&S.bar_mma);
             }
             ok = tc::mbar_wait(&S.bar_mma, (gi + 1) & 1);
             if (__syncthreads_or(!ok)) goto abort;
             tc::tc_fence_after();
-            if (tid == 0 && gi + 1 < G) {   // V buffer is free again: fetch the next head's V
+            if (tid == 0 && gi + 1 < G) {   // the V rows are free again: next head's V
                 tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
-                tc::tma_load_3d(&S.V[0][0], &tm_v, &S.bar_v, 0, h + 1, si);
-                tc::tma_load_3d(&S.V[1][0], &tm_v, &S.bar_v, 64, h + 1, si);
+                tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, h + 1, si);
+                tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, h + 1, si);
             }
-            // ---- epilogue: lane t of D_W / D_U is column t of W / U ----------------------
+            // ---- epilogue: lane t of D_W / D_U is column t of W / U; stage the tiles in
+            //      shared memory, then copy each out as one contiguous 16 KB block ----------
             {
-                float w[64];
-                tc::tmem_ld32(tDW + lane_base, w);
-                tc::tmem_ld32(tDW + lane_base + 32, w + 32);
-                tc::tmem_wait_ld();
-                f16* Wd = Wg + ch * 64 * D + tid;
+                f16* stw = S.AW;                                 // [64][128] fp16 (AW..AU)
+                f16* stu = reinterpret_cast<f16*>(&S.M[0][0]);   // [64][128] fp16
 #pragma unroll
-                for (int i = 0; i < 64; ++i) Wd[i * D] = __float2half_rn(w[i]);
-                tc::tmem_ld32(tDU + lane_base, w);
-                tc::tmem_ld32(tDU + lane_base + 32, w + 32);
-                tc::tmem_wait_ld();
-                float umax = 0.f;
+                for (int part = 0; part < 2; ++part) {
+                    float w[32];
+                    tc::tmem_ld32(tDW + lane_base + part * 32, w);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 64; ++i) umax = fmaxf(umax, fabsf(w[i]));
+                    for (int i = 0; i < 32; ++i) stw[(part * 32 + i) * D + tid] = __float2half_rn(w[i]);
+                    tc::tmem_ld32(tDU + lane_base + part * 32, w);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    umax = fmaxf(umax, __shfl_xor_sync(0xffffffffu, umax, o));
-                    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+                    for (int i = 0; i < 32; ++i) stu[(part * 32 + i) * D + tid] = __float2half_rn(w[i]);
                 }
-                if ((tid & 31) == 0) {
-                    S.red[warp] = umax;
-                    S.red[4 + warp] = vmax;
-                }
+                tc::tc_fence_before();
                 __syncthreads();
-                umax = fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3]));
-                vmax = fmaxf(fmaxf(S.red[4], S.red[5]), fmaxf(S.red[6], S.red[7]));
-                const float uinv = pow2_above(umax), us = 1.f / uinv;   // exact powers of two
-                f16* Ud = Ug + ch * 64 * D + tid;
+                const uint4* sw4 = reinterpret_cast<const uint4*>(stw);
+                const uint4* su4 = reinterpret_cast<const uint4*>(stu);
+                uint4* gw4 = reinterpret_cast<uint4*>(Wg + ch * 64 * D);
+                uint4* gu4 = reinterpret_cast<uint4*>(Ug + ch * 64 * D);
 #pragma unroll
-                for (int i = 0; i < 64; ++i) Ud[i * D] = __float2half_rn(w[i] * us);
-                if (tid == 0) {
-                    SCg[ch * SC_FLOATS + SC_UINV] = uinv;
-                    SCg[ch * SC_FLOATS + SC_VMAX] = vmax;
+                for (int e = tid; e < 64 * D / 8; e += 128) {
+                    gw4[e] = sw4[e];
+                    gu4[e] = su4[e];
                 }
             }
-            tc::tc_fence_before();
             __syncthreads();
         }
     }
@@ -558,12 +558,11 @@ abort:
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kPrepTmemCols);
 }
-
 // ======================================================================================
 // chunk_carry
 // ======================================================================================
 struct CarryStage {
-    f16 A[2][128 * 64];    // [W; Q_hat] in two 64-column halves (32 KB)
+    f16 A[2][128 * 64];    // [W; Q_hat] in two 64-column halves (32 KB), K-major 128B-swizzled
     f16 K[2][64 * 64];     // K_hat in two 64-column halves (16 KB)
     f16 P[128 * 64];       // rows 0-63 zero, rows 64-127 P (16 KB)
     f16 U[64 * NS];        // scaled U columns of this slice, row-major (4 KB)
@@ -571,29 +570,55 @@ struct CarryStage {
 };
 struct CarrySmem {
     CarryStage st[NSTAGE];
-    f16 H0[2][NS * 64];    // scaled fp16 state slice as K-major B operand: rows = value columns
-    f16 Dl[NS * 64];       // scaled Delta as K-major B operand (rows = value columns, K = tokens)
-    f16 Dt[NS * 64];       // scaled Delta~ = diag(exp(G_C - G)) Delta, same layout
+    f16 H0[2][D * NS];     // scaled fp16 state slice: MN-major unswizzled B operand (K = Dk),
+                           //   by chunk parity
+    f16 Dl[C * NS];        // scaled Delta, same layout (K = tokens)
+    f16 Dt[C * NS];        // scaled Delta~ = diag(exp(G_C - G)) Delta
     float red[4];
-    uint64_t full[NSTAGE], empty[NSTAGE], bar_a, bar_bc;
+    uint64_t full[NSTAGE], empty[NSTAGE], bar_a, bar_b, bar_o, h0_ready, d_ready;
     uint32_t tmem_base;
     volatile int abort;
 };
 constexpr size_t kCarrySmemBytes = sizeof(CarrySmem) + 1024;
-constexpr uint32_t kCarryTmemCols = 128;
+constexpr uint32_t kCarryTmemCols = 256;
 constexpr uint32_t kStageTxBytes = 2 * 128 * 64 * 2 + 2 * 64 * 64 * 2 + 64 * 64 * 2 + 64 * NS * 2 + SC_FLOATS * 4;
+constexpr int kCarryThreads = 192;   // warps 0-3 epilogues, warp 4 TMA producer, warp 5 MMA issuer
 
-// store the scaled fp16 copy of state row t (value columns 0..NS-1 of the slice) into
-// the K-major B operand: element (row j, column t)
-__device__ __forceinline__ void store_state_operand(f16* H0, int t, const float* h, float sc) {
-    uint8_t* base = reinterpret_cast<uint8_t*>(H0) + (t >> 6) * (NS * 128);
-    const int c = t & 63;
+// MN-major, unswizzled B operand with N = NS (32) columns: 8 x 8 core matrices of 128 bytes
+// (8 K-rows of 16 bytes); the NS / 8 core matrices of one group of 8 K-rows sit 128 bytes
+// apart (stride between N blocks, SBO), consecutive K groups 512 bytes apart (LBO).
+constexpr uint32_t kOpSBO = 128, kOpLBO = 128 * (NS / 8);
+__device__ __forceinline__ uint32_t op_off(int k, int nb) {   // 16-byte chunk of row k, N block nb
+    return (uint32_t)((k & 7) * 16 + nb * kOpSBO + (k >> 3) * kOpLBO);
+}
+__device__ __forceinline__ uint64_t desc_noswz(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;   // descriptor version; layout bits 61-63 = 0: no swizzle
+    return d;
+}
+// write NS values of row k (scaled, fp16) into an MN-major operand
+__device__ __forceinline__ void store_op_row(f16* op, int k, const float* v, float sc) {
+    uint8_t* base = reinterpret_cast<uint8_t*>(op);
 #pragma unroll
-    for (int j = 0; j < NS; ++j)
-        *reinterpret_cast<f16*>(base + tc::sw128_off(j, c)) = __float2half_rn(h[j] * sc);
+    for (int nb = 0; nb < NS / 8; ++nb) {
+        __align__(16) f16 h8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h8[e] = __float2half_rn(v[nb * 8 + e] * sc);
+        *reinterpret_cast<uint4*>(base + op_off(k, nb)) = *reinterpret_cast<const uint4*>(h8);
+    }
 }
 
-__global__ void __launch_bounds__(160, 1)
+// Per chunk c, the MMA warp issues (each group committed to its own mbarrier):
+//   a: [W; Q_hat] H0     (M=128, 8 MMAs)  -> D_a[c & 1]  rows 0-63 W H0, rows 64-127 Q_hat H0
+//   b: K_hat^T Delta~    (M=128, 4 MMAs)  -> D_b         state update
+//   c: [0; P] Delta      (M=128, 4 MMAs)  -> D_c[c & 1]  rows 64-127 P Delta
+// Epilogue threads 0-63 turn D_a rows into Delta, Delta~; all 128 update the state rows
+// from D_b; threads 64-127 write the output rows of chunk c while chunk c+1's MMAs run.
+// The two sides meet only through mbarriers (h0_ready, d_ready: 128 arrivals each).
+__global__ void __launch_bounds__(kCarryThreads, 1)
 chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qk,
                    const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_u,
                    const float* __restrict__ SCg, const int32_t* __restrict__ cu,
@@ -625,12 +650,15 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
             tc::mbar_init(&S.empty[i], 1);
         }
         tc::mbar_init(&S.bar_a, 1);
-        tc::mbar_init(&S.bar_bc, 1);
+        tc::mbar_init(&S.bar_b, 1);
+        tc::mbar_init(&S.bar_o, 1);
+        tc::mbar_init(&S.h0_ready, 128);
+        tc::mbar_init(&S.d_ready, 128);
         tc::fence_mbar_init();
         S.abort = 0;
     }
     // zero rows 0-63 of the P operands (the producer only ever writes rows 64-127)
-    for (int e = tid; e < NSTAGE * 64 * 64 / 8; e += 160) {
+    for (int e = tid; e < NSTAGE * 64 * 64 / 8; e += kCarryThreads) {
         const int st = e / (64 * 64 / 8), r = e % (64 * 64 / 8);
         reinterpret_cast<uint4*>(S.st[st].P)[r] = make_uint4(0, 0, 0, 0);
     }
@@ -639,6 +667,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = S.tmem_base;
+    const uint32_t tA = tmem, tB = tmem + 64, tC = tmem + 96;   // tA, tC: +32 per chunk parity
 
     if (warp == 4) {
         // ---------------- producer: stream the chunks through the ring ----------------
@@ -648,7 +677,6 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 if (r > 0 && !tc::mbar_wait(&S.empty[st], (r - 1) & 1)) {
                     record_timeout(status);
                     S.abort = 1;
-                    break;
                 }
                 if (S.abort) break;
                 CarryStage& B = S.st[st];
@@ -667,11 +695,54 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 tc::bulk_load(B.SC, SCg + ((size_t)cid * HV + h) * SC_FLOATS, SC_FLOATS * 4, &S.full[st]);
             }
         }
+    } else if (warp == 5) {
+        // ---------------- MMA issuer ---------------------------------------------------------
+        if (lane == 0) {
+            constexpr uint32_t idA = tc::idesc_f16(128, NS, 0, 1);   // K-major A, MN-major B
+            constexpr uint32_t idB = tc::idesc_f16(128, NS, 1, 1);   // MN-major A and B
+            const uint32_t dlb = tc::smem_u32(S.Dl), dtb = tc::smem_u32(S.Dt);
+            for (int c = 0; c < nch; ++c) {
+                const int st = c % NSTAGE, r = c / NSTAGE;
+                const CarryStage& B = S.st[st];
+                bool ok = tc::mbar_wait(&S.full[st], r & 1);
+                ok = ok && tc::mbar_wait(&S.h0_ready, c & 1);
+                if (!ok || S.abort) {
+                    if (!ok) record_timeout(status);
+                    S.abort = 1;
+                    break;
+                }
+                tc::tc_fence_after();
+                const uint32_t par = (uint32_t)(c & 1) * 32;
+                const uint32_t ab = tc::smem_u32(&B.A[0][0]), h0b = tc::smem_u32(S.H0[c & 1]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tA + par, tc::desc_sw128(ab + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                 desc_noswz(h0b + kk * 2 * kOpLBO, kOpLBO, kOpSBO), idA, kk > 0);
+                tc::mma_commit(&S.bar_a);
+                if (!tc::mbar_wait(&S.d_ready, c & 1) || S.abort) {
+                    record_timeout(status);
+                    S.abort = 1;
+                    break;
+                }
+                tc::tc_fence_after();
+                const uint32_t kb = tc::smem_u32(&B.K[0][0]), pb = tc::smem_u32(B.P);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tB, tc::desc_sw128(kb + kk * 2048, 8192, 1024),
+                                 desc_noswz(dtb + kk * 2 * kOpLBO, kOpLBO, kOpSBO), idB, kk > 0);
+                tc::mma_commit(&S.bar_b);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tC + par, tc::desc_sw128(pb + kk * 32, 16, 1024),
+                                 desc_noswz(dlb + kk * 2 * kOpLBO, kOpLBO, kOpSBO), idA, kk > 0);
+                tc::mma_commit(&S.bar_o);
+                tc::mma_commit(&S.empty[st]);   // the stage's operands are consumed
+            }
+        }
     } else {
-        // ---------------- consumers: 128 threads, thread t <-> TMEM lane t -----------------
+        // ---------------- epilogues: 128 threads, thread t <-> TMEM lane t ------------------
         const int t = tid;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const uint32_t tA = tmem, tB = tmem + 32, tC = tmem + 64;
         float Hr[NS];
         const size_t hrow = (((size_t)n * HV + h) * D + t) * D + vs * NS;
         float m = 0.f;
@@ -688,100 +759,96 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         tc::named_bar(1, 128);
         const float inv_sc = pow2_above(fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3])));
         const float sc = 1.f / inv_sc;
-        store_state_operand(&S.H0[0][0], t, Hr, sc);
+        store_op_row(S.H0[0], t, Hr, sc);
         tc::fence_async_smem();
-        tc::named_bar(1, 128);
-        constexpr uint32_t idA = tc::idesc_f16(128, NS, 0, 0);
-        constexpr uint32_t idB = tc::idesc_f16(128, NS, 1, 0);
-        const uint32_t h0b = tc::smem_u32(&S.H0[0][0]);
-        const uint32_t dlb = tc::smem_u32(S.Dl), dtb = tc::smem_u32(S.Dt);
-        bool failed = false;
-        for (int c = 0; c < nch; ++c) {
-            const int st = c % NSTAGE, r = c / NSTAGE;
-            CarryStage& B = S.st[st];
+        tc::mbar_arrive(&S.h0_ready);
+        bool ok = true;
+        float a_prev = 0.f;
+        int cn_prev = 0;
+        int64_t tok_prev = 0;
+        for (int c = 0; c < nch && ok; ++c) {
+            const int st = c % NSTAGE, rr = c / NSTAGE;
+            const CarryStage& B = S.st[st];
             const int64_t tok = bos + (int64_t)C * c;
             const int64_t rem = len - (int64_t)C * c;
             const int cn = (int)(rem < C ? rem : C);
-            bool ok = tc::mbar_wait(&S.full[st], r & 1);
-            if (bar_any(1, 128, !ok)) { failed = true; break; }
-            // ---- D_a = [W; Q] H0 --------------------------------------------------------
-            if (t == 0) {
+            ok = tc::mbar_wait(&S.full[st], rr & 1);
+            // ---- output rows of the previous chunk (threads 64-127) ------------------------
+            if (c > 0 && warp >= 2) {
+                ok = tc::mbar_wait(&S.bar_o, (c - 1) & 1) && ok;
                 tc::tc_fence_after();
-                const uint32_t ab = tc::smem_u32(&B.A[0][0]);
+                const uint32_t par = (uint32_t)((c - 1) & 1) * 32;
+                float q[NS], z[NS];
+                tc::tmem_ld32(tA + par + lane_base, q);
+                tc::tmem_ld32(tC + par + lane_base, z);
+                tc::tmem_wait_ld();
+                if (t - 64 < cn_prev) {
+                    __align__(16) bf16 ob[NS];
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = (kk & 3) * 32;
-                    tc::mma_bf16(tA, tc::desc_sw128(ab + (kk >> 2) * 16384 + koff, 16, 1024),
-                                 tc::desc_sw128(h0b + (kk >> 2) * (NS * 128) + koff, 16, 1024), idA, kk > 0);
+                    for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(a_prev, q[j], z[j]) * inv_sc);
+                    uint4* dst = reinterpret_cast<uint4*>(o + ((tok_prev + t - 64) * HV + h) * D + vs * NS);
+#pragma unroll
+                    for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
                 }
-                tc::mma_commit(&S.bar_a);
             }
-            ok = tc::mbar_wait(&S.bar_a, c & 1);
+            // ---- Delta rows (threads 0-63) ---------------------------------------------------
+            ok = tc::mbar_wait(&S.bar_a, c & 1) && ok;
             tc::tc_fence_after();
-            float x[NS];
-            tc::tmem_ld32(tA + lane_base, x);
-            tc::tmem_wait_ld();
             const float gC = B.SC[SC_GC];
-            float op[NS];
-            if (t < 64) {   // Delta_i = U_i - (W H0)_i ; Delta~_i = d_i Delta_i   (stored scaled)
-                const float di = B.SC[64 + t], uinv = B.SC[SC_UINV];
+            if (warp < 2) {
+                float x[NS];
+                tc::tmem_ld32(tA + (uint32_t)(c & 1) * 32 + lane_base, x);
+                tc::tmem_wait_ld();
+                const float dr = B.SC[64 + t], uinv = B.SC[SC_UINV];
                 const f16* urow = B.U + t * NS;
-                uint8_t* dl = reinterpret_cast<uint8_t*>(S.Dl);
-                uint8_t* dt = reinterpret_cast<uint8_t*>(S.Dt);
+                float dv[NS];
 #pragma unroll
-                for (int j = 0; j < NS; ++j) {
-                    const float dv = __half2float(urow[j]) * uinv - x[j] * inv_sc;
-                    const uint32_t off = tc::sw128_off(j, t);
-                    *reinterpret_cast<f16*>(dl + off) = __float2half_rn(dv * sc);
-                    *reinterpret_cast<f16*>(dt + off) = __float2half_rn(di * dv * sc);
-                }
-            } else {        // the inter-chunk part of the output rows
-                const float ai = B.SC[t - 64] * inv_sc;
-#pragma unroll
-                for (int j = 0; j < NS; ++j) op[j] = ai * x[j];
+                for (int j = 0; j < NS; ++j) dv[j] = __half2float(urow[j]) * uinv - x[j] * inv_sc;
+                store_op_row(S.Dl, t, dv, sc);
+                store_op_row(S.Dt, t, dv, dr * sc);
+                tc::fence_async_smem();
+            } else {
+                a_prev = B.SC[t - 64];
             }
+            cn_prev = cn;
+            tok_prev = tok;
             tc::tc_fence_before();
-            tc::fence_async_smem();
-            if (bar_any(1, 128, !ok)) { failed = true; break; }
-            // ---- D_b = K^T Delta~ (state update), D_c = [0; P] Delta (output) ------------
-            if (t == 0) {
-                tc::tc_fence_after();
-                const uint32_t kb = tc::smem_u32(&B.K[0][0]);
-                const uint32_t pb = tc::smem_u32(B.P);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tB, tc::desc_sw128(kb + kk * 2048, 8192, 1024),
-                                 tc::desc_sw128(dtb + kk * 32, 16, 1024), idB, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tC, tc::desc_sw128(pb + kk * 32, 16, 1024),
-                                 tc::desc_sw128(dlb + kk * 32, 16, 1024), idA, kk > 0);
-                tc::mma_commit(&S.bar_bc);
-                tc::mma_commit(&S.empty[st]);   // the stage's operands are consumed
-            }
-            ok = tc::mbar_wait(&S.bar_bc, c & 1);
+            tc::mbar_arrive(&S.d_ready);
+            // ---- state rows (all 128) ---------------------------------------------------------
+            ok = tc::mbar_wait(&S.bar_b, c & 1) && ok;
             tc::tc_fence_after();
-            float y[NS];
-            tc::tmem_ld32(tB + lane_base, y);
-            if (warp >= 2) tc::tmem_ld32(tC + lane_base, x);
-            tc::tmem_wait_ld();
+            {
+                float y[NS];
+                tc::tmem_ld32(tB + lane_base, y);
+                tc::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < NS; ++j) Hr[j] = fmaf(gC, Hr[j], y[j] * inv_sc);
-            store_state_operand(&S.H0[0][0], t, Hr, sc);
-            if (t >= 64 && t - 64 < cn) {
+                for (int j = 0; j < NS; ++j) Hr[j] = fmaf(gC, Hr[j], y[j] * inv_sc);
+            }
+            store_op_row(S.H0[(c + 1) & 1], t, Hr, sc);
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&S.h0_ready);
+            if (S.abort) ok = false;
+        }
+        if (ok && nch > 0 && warp >= 2) {   // output rows of the last chunk
+            ok = tc::mbar_wait(&S.bar_o, (nch - 1) & 1);
+            tc::tc_fence_after();
+            const uint32_t par = (uint32_t)((nch - 1) & 1) * 32;
+            float q[NS], z[NS];
+            tc::tmem_ld32(tA + par + lane_base, q);
+            tc::tmem_ld32(tC + par + lane_base, z);
+            tc::tmem_wait_ld();
+            if (ok && t - 64 < cn_prev) {
                 __align__(16) bf16 ob[NS];
 #pragma unroll
-                for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(x[j], inv_sc, op[j]));
-                uint4* dst = reinterpret_cast<uint4*>(o + ((tok + t - 64) * HV + h) * D + vs * NS);
+                for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(a_prev, q[j], z[j]) * inv_sc);
+                uint4* dst = reinterpret_cast<uint4*>(o + ((tok_prev + t - 64) * HV + h) * D + vs * NS);
 #pragma unroll
-                for (int q = 0; q < NS / 8; ++q) dst[q] = reinterpret_cast<const uint4*>(ob)[q];
+                for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
             }
-            tc::tc_fence_before();
-            tc::fence_async_smem();
-            if (bar_any(1, 128, !ok)) { failed = true; break; }
         }
-        if (failed) {
-            if (t == 0) record_timeout(status);
+        if (!ok) {
+            record_timeout(status);
             S.abort = 1;
         } else if (hT) {
 #pragma unroll
@@ -948,7 +1015,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
     e = cudaFuncSetAttribute(chunk_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCarrySmemBytes);
     if (e != cudaSuccess) return e;
     const unsigned blocks = (unsigned)a.n_seqs * (unsigned)a.HV * (unsigned)(D / NS);
-    chunk_carry_kernel<<<blocks, 160, kCarrySmemBytes, s>>>(tw, tqk, tp, tu, SC, a.cu, chunk_off, a.T, a.n_seqs,
+    chunk_carry_kernel<<<blocks, kCarryThreads, kCarrySmemBytes, s>>>(tw, tqk, tp, tu, SC, a.cu, chunk_off, a.T, a.n_seqs,
                                                           a.HK, a.HV, a.h0, a.hT, (bf16*)a.o, a.status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

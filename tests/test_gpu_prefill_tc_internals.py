@@ -1,6 +1,6 @@
 """White-box check of the tensor-core prefill's chunk-local stage: after a call,
 the workspace holds, per (chunk, value head), fp16 W = T diag(b gamma) K_hat,
-U = T diag(b) V (stored as fp16(U / 2^e) with 2^e alongside),
+U = T diag(b) V (stored as fp16(U / 2^e) with 2^e alongside, e from max|v|),
 P = scale * (exp(G_i - G_j) q_hat_i . k_hat_j)_{i>=j}, the per-row scalars, and per
 (chunk, q/k head) the normalised fp16 K_hat and Q_hat tiles.  They are recomputed
 here in numpy fp64 from the same inputs (the gates from the oracle) and compared at
@@ -93,7 +93,7 @@ def test_chunk_local_stage(HK, HV):
             np.testing.assert_allclose(SC[c, h, 64:64 + cn], d_ref, rtol=1e-4, err_msg=tag + " d")
             np.testing.assert_allclose(SC[c, h, 128], np.exp(Gc[-1]), rtol=1e-4, err_msg=tag + " gC")
             np.testing.assert_allclose(SC[c, h, 130], np.abs(V).max(), rtol=1e-6, err_msg=tag + " vmax")
-            assert 0.5 <= np.abs(U_ref).max() / SC[c, h, 129] < 1.0
+            assert 0.5 <= np.abs(V).max() / SC[c, h, 129] < 1.0   # U is stored as fp16(U * 2^-e) with max|v| * 2^-e in [0.5, 1)
             assert np.all(W[c, h, cn:] == 0) and np.all(U[c, h, cn:] == 0)
             if h % Gq == 0:
                 np.testing.assert_allclose(QK[c, hk, :cn], Kh, atol=2e-3 * np.abs(Kh).max(), err_msg=tag + " K_hat")
