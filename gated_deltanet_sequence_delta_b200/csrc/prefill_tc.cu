@@ -157,51 +157,95 @@ __global__ void __launch_bounds__(1024) chunk_table_kernel(const int32_t* __rest
 // implied); entries on and above the diagonal are untouched.  Blocks of 16:
 //  * diagonal blocks T_bb = (I + L_bb)^-1 by right-looking column substitution: every
 //    finished x_j updates all later rows at once, so the dependent chain is one FMA per row;
-//  * block rows I = 1, 2, 3: T_Ij = -T_II sum_{k=j}^{I-1} L_Ik T_kj for all j < I at once.
-//    Row block I of L is read only while row block I of T is formed, so T overwrites it.
+//  * block rows I = 1, 2, 3: T_Ij = -T_II sum_{k=j}^{I-1} L_Ik T_kj for all j < I at once,
+//    one warp per j, the 16 x 16 block products on mma.sync with fp16 operands (the T
+//    entries are rounded to fp16 for the W / U operands anyway).  Row block I of L is
+//    read only while row block I of T is formed, so T overwrites it.
 // ======================================================================================
+// Warp-level 16x16x16 products on the legacy tensor-core path (mma.sync m16n8k16, fp16
+// operands, fp32 accumulation); fragment layouts of that instruction: g = lane / 4,
+// q = lane % 4; A (16 x 16): rows g, g+8 x columns 2q, 2q+1, 2q+8, 2q+9; B (16 x 8):
+// rows 2q, 2q+1, 2q+8, 2q+9 x column g; D (16 x 8): rows g, g+8 x columns 2q, 2q+1.
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// Element (r, c) of a 16 x 16 block of M at (r0, c0); UNIT: the block is a diagonal block
+// of T (unit diagonal implied, zero above it).
+template <bool UNIT>
+__device__ __forceinline__ float blk(const float (*M)[65], int r0, int c0, int r, int c) {
+    if (UNIT) return r == c ? 1.f : (r > c ? M[r0 + r][c0 + c] : 0.f);
+    return M[r0 + r][c0 + c];
+}
+template <bool UNIT>
+__device__ __forceinline__ void frag_a(uint32_t* a, const float (*M)[65], int r0, int c0, int g, int q) {
+    a[0] = pack_h2(blk<UNIT>(M, r0, c0, g, 2 * q), blk<UNIT>(M, r0, c0, g, 2 * q + 1));
+    a[1] = pack_h2(blk<UNIT>(M, r0, c0, g + 8, 2 * q), blk<UNIT>(M, r0, c0, g + 8, 2 * q + 1));
+    a[2] = pack_h2(blk<UNIT>(M, r0, c0, g, 2 * q + 8), blk<UNIT>(M, r0, c0, g, 2 * q + 9));
+    a[3] = pack_h2(blk<UNIT>(M, r0, c0, g + 8, 2 * q + 8), blk<UNIT>(M, r0, c0, g + 8, 2 * q + 9));
+}
+// B fragment of the 16 x 8 slice (all 16 rows, columns n0 .. n0+7) of a block
+template <bool UNIT>
+__device__ __forceinline__ void frag_b(uint32_t* b, const float (*M)[65], int r0, int c0, int n0, int g, int q) {
+    b[0] = pack_h2(blk<UNIT>(M, r0, c0, 2 * q, n0 + g), blk<UNIT>(M, r0, c0, 2 * q + 1, n0 + g));
+    b[1] = pack_h2(blk<UNIT>(M, r0, c0, 2 * q + 8, n0 + g), blk<UNIT>(M, r0, c0, 2 * q + 9, n0 + g));
+}
+
+// Block row I of T: warp j (< I) forms X_j = sum_{k=j}^{I-1} L_Ik T_kj, then T_Ij = -T_II X_j.
 template <int I>
 __device__ __forceinline__ void tinv_row_block(float (*M)[65], float (*X)[16][17], int tid) {
-    const int c = tid & 15, r0 = tid >> 4;   // this thread: rows r0 and r0 + 8, column c
-    float acc[I][2];
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+    const float(*Xc)[17] = nullptr;
+    if (warp < I) {
+        const int j = warp;
+        float acc[2][4] = {};
 #pragma unroll
-    for (int j = 0; j < I; ++j) acc[j][0] = acc[j][1] = 0.f;
+        for (int k = 0; k < I; ++k) {
+            if (k < j) continue;
+            uint32_t a[4], b[2];
+            frag_a<false>(a, M, 16 * I, 16 * k, g, q);
 #pragma unroll
-    for (int j = 0; j < I; ++j) {
-#pragma unroll
-        for (int k = j; k < I; ++k) {
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-                float t;
-                if (k == j) t = kk == c ? 1.f : (kk > c ? M[16 * j + kk][16 * j + c] : 0.f);
-                else t = M[16 * k + kk][16 * j + c];
-                acc[j][0] = fmaf(M[16 * I + r0][16 * k + kk], t, acc[j][0]);
-                acc[j][1] = fmaf(M[16 * I + r0 + 8][16 * k + kk], t, acc[j][1]);
+            for (int nt = 0; nt < 2; ++nt) {
+                if (k == j) frag_b<true>(b, M, 16 * k, 16 * j, 8 * nt, g, q);
+                else frag_b<false>(b, M, 16 * k, 16 * j, 8 * nt, g, q);
+                mma16816(acc[nt], a, b);
             }
         }
-    }
 #pragma unroll
-    for (int j = 0; j < I; ++j) {
-        X[j][r0][c] = acc[j][0];
-        X[j][r0 + 8][c] = acc[j][1];
+        for (int nt = 0; nt < 2; ++nt) {
+            X[j][g][8 * nt + 2 * q] = acc[nt][0];
+            X[j][g][8 * nt + 2 * q + 1] = acc[nt][1];
+            X[j][g + 8][8 * nt + 2 * q] = acc[nt][2];
+            X[j][g + 8][8 * nt + 2 * q + 1] = acc[nt][3];
+        }
     }
     __syncthreads();   // every read of row block I of L is done before it is overwritten
+    if (warp < I) {
+        const int j = warp;
+        Xc = X[j];
+        float acc[2][4] = {};
+        uint32_t a[4], b[2];
+        frag_a<true>(a, M, 16 * I, 16 * I, g, q);
 #pragma unroll
-    for (int j = 0; j < I; ++j) {
-        float a0 = X[j][r0][c], a1 = X[j][r0 + 8][c];
-#pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
-            const float xk = X[j][kk][c];
-            if (kk < r0) a0 = fmaf(M[16 * I + r0][16 * I + kk], xk, a0);
-            if (kk < r0 + 8) a1 = fmaf(M[16 * I + r0 + 8][16 * I + kk], xk, a1);
+        for (int nt = 0; nt < 2; ++nt) {
+            b[0] = pack_h2(Xc[2 * q][8 * nt + g], Xc[2 * q + 1][8 * nt + g]);
+            b[1] = pack_h2(Xc[2 * q + 8][8 * nt + g], Xc[2 * q + 9][8 * nt + g]);
+            mma16816(acc[nt], a, b);
         }
-        acc[j][0] = -a0;
-        acc[j][1] = -a1;
-    }
 #pragma unroll
-    for (int j = 0; j < I; ++j) {
-        M[16 * I + r0][16 * j + c] = acc[j][0];
-        M[16 * I + r0 + 8][16 * j + c] = acc[j][1];
+        for (int nt = 0; nt < 2; ++nt) {
+            M[16 * I + g][16 * j + 8 * nt + 2 * q] = -acc[nt][0];
+            M[16 * I + g][16 * j + 8 * nt + 2 * q + 1] = -acc[nt][1];
+            M[16 * I + g + 8][16 * j + 8 * nt + 2 * q] = -acc[nt][2];
+            M[16 * I + g + 8][16 * j + 8 * nt + 2 * q + 1] = -acc[nt][3];
+        }
     }
     __syncthreads();
 }
@@ -322,8 +366,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int half = 0; half < 2; ++half) {
             const uint4* row = reinterpret_cast<const uint4*>(kq + half * 16384 + tid * 128);
 #pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
-                const uint4 u = row[c16];
+            for (int c16 = 0; c16 < 8; ++c16) {   // chunk order c16 ^ (row % 8): conflict-free
+                const uint4 u = row[c16 ^ (tid & 7)];
                 const bf16* e = reinterpret_cast<const bf16*>(&u);
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
@@ -407,7 +451,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     float v = 0.f;
-                    if (j < i && i < cn) v = bi * expf(Gi - S.G[j]) * S.rk[j] * row[j];
+                    if (j < i && i < cn) v = bi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
                     S.M[i][j] = v;
                 }
                 SCg[ch * SC_FLOATS + 64 + i] = i < cn ? expf(Gl - Gi) : 0.f;
@@ -424,7 +468,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int t = 0; t < 8; ++t) {
                         const int j = c8 * 8 + t;
                         float v = 0.f;
-                        if (j <= i && i < cn) v = qi * expf(Gi - S.G[j]) * S.rk[j] * row[j];
+                        if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
                         e[t] = __float2half_rn(v);
                     }
                     prow[c8] = *reinterpret_cast<const uint4*>(e);
@@ -463,7 +507,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (r < cn) {
 #pragma unroll
                     for (int c16 = 0; c16 < 8; ++c16) {
-                        const uint4 u = vr[c16];
+                        const uint4 u = vr[c16 ^ (r & 7)];
                         const bf16* e = reinterpret_cast<const bf16*>(&u);
 #pragma unroll
                         for (int t = 0; t < 8; ++t) vmax = fmaxf(vmax, fabsf(__bfloat162float(e[t])));
@@ -477,12 +521,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const float uinv = pow2_above(vmax), sv = r < cn ? 1.f / uinv : 0.f;
 #pragma unroll
                 for (int c16 = 0; c16 < 8; ++c16) {
-                    const uint4 u = vr[c16];
+                    const int pc = c16 ^ (r & 7);
+                    const uint4 u = vr[pc];
                     const bf16* e = reinterpret_cast<const bf16*>(&u);
                     __align__(16) f16 hx[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) hx[t] = __float2half_rn(__bfloat162float(e[t]) * sv);
-                    vr[c16] = *reinterpret_cast<const uint4*>(hx);
+                    vr[pc] = *reinterpret_cast<const uint4*>(hx);
                 }
                 if (tid == 0) {
                     SCg[ch * SC_FLOATS + SC_UINV] = uinv;
@@ -800,10 +845,17 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 tc::tmem_ld32(tA + (uint32_t)(c & 1) * 32 + lane_base, x);
                 tc::tmem_wait_ld();
                 const float dr = B.SC[64 + t], uinv = B.SC[SC_UINV];
-                const f16* urow = B.U + t * NS;
+                const uint4* urow = reinterpret_cast<const uint4*>(B.U + t * NS);
                 float dv[NS];
 #pragma unroll
-                for (int j = 0; j < NS; ++j) dv[j] = __half2float(urow[j]) * uinv - x[j] * inv_sc;
+                for (int nb = 0; nb < NS / 8; ++nb) {   // 16-byte pieces of the row
+                    const uint4 u = urow[nb];
+                    const f16* e = reinterpret_cast<const f16*>(&u);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) dv[nb * 8 + q] = __half2float(e[q]) * uinv;
+                }
+#pragma unroll
+                for (int j = 0; j < NS; ++j) dv[j] -= x[j] * inv_sc;
                 store_op_row(S.Dl, t, dv, sc);
                 store_op_row(S.Dt, t, dv, dr * sc);
                 tc::fence_async_smem();
