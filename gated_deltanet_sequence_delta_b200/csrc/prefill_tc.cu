@@ -662,7 +662,10 @@ __device__ __forceinline__ void store_op_row(f16* op, int k, const float* v, flo
 //   c: [0; P] Delta      (M=128, 4 MMAs)  -> D_c[c & 1]  rows 64-127 P Delta
 // Epilogue threads 0-63 turn D_a rows into Delta, Delta~; all 128 update the state rows
 // from D_b; threads 64-127 write the output rows of chunk c while chunk c+1's MMAs run.
-// The two sides meet only through mbarriers (h0_ready, d_ready: 128 arrivals each).
+// The two sides meet only through mbarriers (h0_ready, d_ready: 128 arrivals each; the
+// output threads arrive on d_ready as soon as they have read the chunk's scalars, then
+// write the previous chunk's output rows while Delta and the state MMA proceed; the
+// stage is released only after every thread's reads of it).
 __global__ void __launch_bounds__(kCarryThreads, 1)
 chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qk,
                    const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_u,
@@ -745,7 +748,8 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         if (lane == 0) {
             constexpr uint32_t idA = tc::idesc_f16(128, NS, 0, 1);   // K-major A, MN-major B
             constexpr uint32_t idB = tc::idesc_f16(128, NS, 1, 1);   // MN-major A and B
-            const uint32_t dlb = tc::smem_u32(S.Dl), dtb = tc::smem_u32(S.Dt);
+            const uint64_t ddl = desc_noswz(tc::smem_u32(S.Dl), kOpLBO, kOpSBO);
+            const uint64_t ddt = desc_noswz(tc::smem_u32(S.Dt), kOpLBO, kOpSBO);
             for (int c = 0; c < nch; ++c) {
                 const int st = c % NSTAGE, r = c / NSTAGE;
                 const CarryStage& B = S.st[st];
@@ -758,11 +762,13 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 }
                 tc::tc_fence_after();
                 const uint32_t par = (uint32_t)(c & 1) * 32;
-                const uint32_t ab = tc::smem_u32(&B.A[0][0]), h0b = tc::smem_u32(S.H0[c & 1]);
+                // descriptors built once; a k-step only advances the start-address field
+                const uint64_t da = tc::desc_sw128(tc::smem_u32(&B.A[0][0]), 16, 1024);
+                const uint64_t dh = desc_noswz(tc::smem_u32(S.H0[c & 1]), kOpLBO, kOpSBO);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(tA + par, tc::desc_sw128(ab + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                 desc_noswz(h0b + kk * 2 * kOpLBO, kOpLBO, kOpSBO), idA, kk > 0);
+                    tc::mma_bf16(tA + par, da + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                 dh + (uint64_t)((kk * 2 * kOpLBO) >> 4), idA, kk > 0);
                 tc::mma_commit(&S.bar_a);
                 if (!tc::mbar_wait(&S.d_ready, c & 1) || S.abort) {
                     record_timeout(status);
@@ -770,16 +776,17 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                     break;
                 }
                 tc::tc_fence_after();
-                const uint32_t kb = tc::smem_u32(&B.K[0][0]), pb = tc::smem_u32(B.P);
+                const uint64_t dk = tc::desc_sw128(tc::smem_u32(&B.K[0][0]), 8192, 1024);
+                const uint64_t dp = tc::desc_sw128(tc::smem_u32(B.P), 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tB, tc::desc_sw128(kb + kk * 2048, 8192, 1024),
-                                 desc_noswz(dtb + kk * 2 * kOpLBO, kOpLBO, kOpSBO), idB, kk > 0);
+                    tc::mma_bf16(tB, dk + (uint64_t)((kk * 2048) >> 4), ddt + (uint64_t)((kk * 2 * kOpLBO) >> 4),
+                                 idB, kk > 0);
                 tc::mma_commit(&S.bar_b);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tC + par, tc::desc_sw128(pb + kk * 32, 16, 1024),
-                                 desc_noswz(dlb + kk * 2 * kOpLBO, kOpLBO, kOpSBO), idA, kk > 0);
+                    tc::mma_bf16(tC + par, dp + (uint64_t)((kk * 32) >> 4), ddl + (uint64_t)((kk * 2 * kOpLBO) >> 4),
+                                 idA, kk > 0);
                 tc::mma_commit(&S.bar_o);
                 tc::mma_commit(&S.empty[st]);   // the stage's operands are consumed
             }
@@ -818,29 +825,11 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
             const int64_t rem = len - (int64_t)C * c;
             const int cn = (int)(rem < C ? rem : C);
             ok = tc::mbar_wait(&S.full[st], rr & 1);
-            // ---- output rows of the previous chunk (threads 64-127) ------------------------
-            if (c > 0 && warp >= 2) {
-                ok = tc::mbar_wait(&S.bar_o, (c - 1) & 1) && ok;
-                tc::tc_fence_after();
-                const uint32_t par = (uint32_t)((c - 1) & 1) * 32;
-                float q[NS], z[NS];
-                tc::tmem_ld32(tA + par + lane_base, q);
-                tc::tmem_ld32(tC + par + lane_base, z);
-                tc::tmem_wait_ld();
-                if (t - 64 < cn_prev) {
-                    __align__(16) bf16 ob[NS];
-#pragma unroll
-                    for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(a_prev, q[j], z[j]) * inv_sc);
-                    uint4* dst = reinterpret_cast<uint4*>(o + ((tok_prev + t - 64) * HV + h) * D + vs * NS);
-#pragma unroll
-                    for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
-                }
-            }
-            // ---- Delta rows (threads 0-63) ---------------------------------------------------
-            ok = tc::mbar_wait(&S.bar_a, c & 1) && ok;
-            tc::tc_fence_after();
             const float gC = B.SC[SC_GC];
             if (warp < 2) {
+                // ---- Delta rows (threads 0-63) ----------------------------------------------
+                ok = tc::mbar_wait(&S.bar_a, c & 1) && ok;
+                tc::tc_fence_after();
                 float x[NS];
                 tc::tmem_ld32(tA + (uint32_t)(c & 1) * 32 + lane_base, x);
                 tc::tmem_wait_ld();
@@ -859,13 +848,34 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 store_op_row(S.Dl, t, dv, sc);
                 store_op_row(S.Dt, t, dv, dr * sc);
                 tc::fence_async_smem();
+                tc::tc_fence_before();
+                tc::mbar_arrive(&S.d_ready);
             } else {
-                a_prev = B.SC[t - 64];
+                // ---- output rows of the previous chunk (threads 64-127), under this chunk's
+                //      Delta epilogue and state MMA -------------------------------------------
+                const float a_cur = B.SC[t - 64];
+                tc::mbar_arrive(&S.d_ready);   // the stage's scalars are read
+                if (c > 0) {
+                    ok = tc::mbar_wait(&S.bar_o, (c - 1) & 1) && ok;
+                    tc::tc_fence_after();
+                    const uint32_t par = (uint32_t)((c - 1) & 1) * 32;
+                    float q[NS], z[NS];
+                    tc::tmem_ld32(tA + par + lane_base, q);
+                    tc::tmem_ld32(tC + par + lane_base, z);
+                    tc::tmem_wait_ld();
+                    if (t - 64 < cn_prev) {
+                        __align__(16) bf16 ob[NS];
+#pragma unroll
+                        for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(a_prev, q[j], z[j]) * inv_sc);
+                        uint4* dst = reinterpret_cast<uint4*>(o + ((tok_prev + t - 64) * HV + h) * D + vs * NS);
+#pragma unroll
+                        for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
+                    }
+                }
+                a_prev = a_cur;
             }
             cn_prev = cn;
             tok_prev = tok;
-            tc::tc_fence_before();
-            tc::mbar_arrive(&S.d_ready);
             // ---- state rows (all 128) ---------------------------------------------------------
             ok = tc::mbar_wait(&S.bar_b, c & 1) && ok;
             tc::tc_fence_after();
