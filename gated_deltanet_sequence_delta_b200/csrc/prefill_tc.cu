@@ -73,20 +73,6 @@ __device__ __forceinline__ void record_timeout(int32_t* status) {
     atomicCAS(status, GDN_DEVERR_NONE, GDN_DEVERR_TIMEOUT);
 }
 
-// true if any of the n threads meeting at barrier `id` passes pred = true
-__device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(n)
-        : "memory");
-    return r != 0;
-}
-
 // Locate chunk `chunk` of the flattened chunk list: its sequence n, first token s and
 // length cn.  chunk_off[n] is the first chunk of sequence n (chunk_off[N] = total).
 __device__ __forceinline__ bool locate_chunk(int chunk, const int32_t* __restrict__ chunk_off,
