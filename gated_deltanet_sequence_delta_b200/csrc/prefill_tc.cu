@@ -19,18 +19,19 @@
 //
 // Precision.  The output is a sum of terms much larger than itself (U - W H0 cancels, so
 // does P Delta against the decayed Q H0 part), so bf16 rounding of the intermediates
-// alone costs 3-5% of RMS(o).  Hence: the chunk-local products W and U are formed with
-// the T operands split into bf16 hi + lo parts against the exact bf16 inputs, and every
-// intermediate operand of the serial stage is fp16 (10-bit mantissa).  Data-dependent
-// operands (state, Delta, U) carry a power-of-two scale so fp16 range is never at issue.
+// alone costs 3-5% of RMS(o).  Hence every intermediate operand is fp16 (10-bit
+// mantissa): the normalised K_hat, Q_hat, the T diag(.) factors and V of the chunk-local
+// products, and W, U, P, Delta and the state copy of the serial stage.  Data-dependent
+// operands (V, U, Delta, state) carry a power-of-two scale so fp16 range is never at issue.
 //
 // Two kernels:
-//  * chunk_prep (one CTA per chunk and q/k head, fully parallel): the Gram tiles
-//    [K;Q] K^T on tcgen05 (M=128), norms, gates, the unit-lower-triangular inverse T in
-//    fp32 on CUDA cores (16x16 diagonal blocks by substitution, off-diagonal blocks by
-//    block products), then W^T = K^T (T diag(b gamma rk))^T and U^T = V^T (T diag(b))^T on
-//    tcgen05 (M=128: Dk or Dv rows).  Writes fp16 W, U (scaled), P, the normalised fp16
-//    K_hat, Q_hat tiles and per-row scalars.
+//  * chunk_prep (one CTA per chunk and q/k head, fully parallel, four CTAs per SM): the
+//    Gram tiles [K;Q] K^T on tcgen05 (M=128), norms, gates, the unit-lower-triangular
+//    inverse T in fp32 (16x16 diagonal blocks by substitution, off-diagonal blocks by
+//    mma.sync block products), then W^T = K_hat^T (T diag(b gamma))^T and
+//    U^T = V^T (T diag(b))^T on tcgen05 (M=128: Dk or Dv rows), read out of TMEM straight
+//    to global memory.  Writes fp16 W, U (scaled), P, the normalised fp16 K_hat, Q_hat
+//    tiles and per-row scalars.
 //  * chunk_carry (one CTA per sequence, value head and 32-column slice of Dv; the value
 //    columns of the state evolve independently): walks the chunks in order.  Per chunk:
 //    [W;Q_hat] H0 (M=128) -> Delta on CUDA cores -> K_hat^T Delta~ and [0;P] Delta (M=128),
@@ -269,20 +270,43 @@ struct PrepSmem {
     // rewritten in place as fp16 K_hat; rows 64-127 are reused for V (bf16 from TMA, then
     // fp16 V * sv in place) once Q_hat has been written out.
     uint16_t KQ[2][128 * 64];
-    f16 AW[64 * 64];        // T diag(b gamma) as K-major B operand (rows i, K = j); later
-    f16 AU[64 * 64];        //   AW..AU stage the fp16 W tile on its way to global memory
-    float M[64][65];        // L, then T in place; later stages the U tile
+    // L, then T in place (fp32, row stride 65); then, in the same bytes, the fp16 MMA
+    // operands T diag(b gamma) (bytes 0-8191) and T diag(b) (8192-16383), K-major 128B-swizzled
+    float M[64][65];
     float X[3][16][17];
     float rk[64], rq[64], G[64], bt[64], bgr[64], red[8];
     float ga[2][64], ba[2][64];   // prefetched g, beta of the (up to two) value heads
     uint64_t bar_load, bar_v, bar_mma;
     uint32_t tmem_base;
 };
+static_assert(offsetof(PrepSmem, M) % 1024 == 0, "the swizzled operands in M need 1024-byte alignment");
 constexpr size_t kPrepSmemBytes = sizeof(PrepSmem) + 1024;
-constexpr uint32_t kPrepTmemCols = 128;
+constexpr uint32_t kPrepTmemCols = 128;   // 4 resident CTAs fill the 512 columns
+
+// Column t = tid of a 64 x 128 fp16 tile from TMEM lane t (64 fp32 columns = the tile's 64
+// rows), stored straight to global memory.  Lane pairs swap one value so that each thread
+// writes 4-byte pairs: per warp and row, 64 contiguous bytes.
+__device__ __forceinline__ void store_tile_from_tmem(f16* __restrict__ dst, uint32_t taddr, int tid) {
+    const bool odd = (tid & 1) != 0;
+    const int col = tid - (odd ? 1 : 0);
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        float w[32];
+        tc::tmem_ld32(taddr + part * 32, w);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+            const float send = odd ? w[2 * p] : w[2 * p + 1];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+            const int row = part * 32 + 2 * p + (odd ? 1 : 0);
+            const __half2 h = odd ? __floats2half2_rn(recv, w[2 * p + 1]) : __floats2half2_rn(w[2 * p], recv);
+            *reinterpret_cast<__half2*>(dst + (size_t)row * D + col) = h;
+        }
+    }
+}
 
 template <int G>
-__global__ void __launch_bounds__(128, 3)
+__global__ void __launch_bounds__(128, 4)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
                   const float* __restrict__ beta, const int32_t* __restrict__ cu,
@@ -313,9 +337,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc::tc_fence_after();
     const uint32_t tmem = S.tmem_base;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t tD1 = tmem, tDU = tmem, tDW = tmem + 64;   // D_U reuses D1's columns
+    // TMEM: columns 0-63 the Gram tiles (kept for every value head), 64-127 W^T; U^T goes
+    // to 64-127 after W^T is read out, except for the last value head, whose U^T takes the
+    // Gram columns (no longer needed) so both products run back to back.
+    const uint32_t tG = tmem, tW = tmem + 64;
     const int si = (int)s;
     uint8_t* kq = reinterpret_cast<uint8_t*>(&S.KQ[0][0]);
+    uint32_t mma_phase = 0;
 
     if (tid == 0) {
         tc::mbar_expect_tx(&S.bar_load, 4 * 64 * 64 * 2);
@@ -335,18 +363,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     bool ok = tc::mbar_wait(&S.bar_load, 0);
     if (__syncthreads_or(!ok)) goto abort;
 
-    // ---- Gram tiles: D1[0:64] = K K^T, D1[64:128] = Q K^T (bf16, M=128, N=64, K=Dk) ----
+    // ---- Gram tiles: D_G[0:64] = K K^T, D_G[64:128] = Q K^T (bf16, M=128, N=64, K=Dk) ----
     if (tid == 0) {
         tc::tc_fence_after();
         const uint32_t base = tc::smem_u32(kq);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint64_t d = tc::desc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            tc::mma_bf16(tD1, d, d, tc::idesc_bf16(128, 64, 0, 0), kk > 0);
+            tc::mma_bf16(tG, d, d, tc::idesc_bf16(128, 64, 0, 0), kk > 0);
         }
         tc::mma_commit(&S.bar_mma);
     }
-    if (tid >= 64) {   // inverse norms of q rows (order inside a row is irrelevant)
+    {   // inverse norms of the k (tid < 64) and q rows, under the Gram MMA (order inside a
+        // row is irrelevant)
         float ss = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -362,24 +391,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
         }
-        S.rq[tid - 64] = l2_inv(ss, l2norm);
+        if (tid < 64) S.rk[tid] = l2_inv(ss, l2norm);
+        else S.rq[tid - 64] = l2_inv(ss, l2norm);
     }
-    ok = tc::mbar_wait(&S.bar_mma, 0);
+    ok = tc::mbar_wait(&S.bar_mma, mma_phase);
+    mma_phase ^= 1;
     if (__syncthreads_or(!ok)) goto abort;
     tc::tc_fence_after();
     {
-        float row[64];
-        tc::tmem_ld32(tD1 + lane_base, row);
-        tc::tmem_ld32(tD1 + lane_base + 32, row + 32);
-        tc::tmem_wait_ld();
-        if (tid < 64) {
-            float diag = 0.f;
-#pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (j == tid) diag = row[j];
-            S.rk[tid] = l2_inv(diag, l2norm);   // k.k from the Gram diagonal
-        }
-        __syncthreads();
         const float rki = tid < 64 ? S.rk[tid] : 0.f;
         const float rqi = tid >= 64 ? S.rq[tid - 64] : 0.f;
         {   // K_hat (tid < 64) / Q_hat row: fp16 in place (K_hat feeds the W MMA) and out to
@@ -414,6 +433,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int gi = 0; gi < G; ++gi) {
             const int h = hk * G + gi;
             const size_t ch = (size_t)chunk * HV + h;
+            const bool last = gi == G - 1;
             // ---- running sum of the log-decays, write strengths -------------------------
             if (tid < 64) {
                 float gv = S.ga[gi][tid];
@@ -430,52 +450,66 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncthreads();
             if (tid < 64) S.bgr[tid] = S.bt[tid] * expf(S.G[tid]);
             const float Gl = S.G[63];   // padding adds 0, so this is G at the last token
-            // ---- L (strictly lower) into M, P (lower incl. diagonal) out, scalars ------
-            if (tid < 64) {
-                const int i = tid;
-                const float Gi = S.G[i], bi = S.bt[i] * rki;
+            // ---- L (strictly lower) into M, P (lower incl. diagonal) out, scalars; the
+            //      Gram row of this thread is read back from TMEM --------------------------
+            {
+                float row[64];
+                tc::tmem_ld32(tG + lane_base, row);
+                tc::tmem_ld32(tG + lane_base + 32, row + 32);
+                tc::tmem_wait_ld();
+                if (tid < 64) {
+                    const int i = tid;
+                    const float Gi = S.G[i], bi = S.bt[i] * rki;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    float v = 0.f;
-                    if (j < i && i < cn) v = bi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
-                    S.M[i][j] = v;
-                }
-                SCg[ch * SC_FLOATS + 64 + i] = i < cn ? expf(Gl - Gi) : 0.f;
-            } else {
-                const int i = tid - 64;
-                const float Gi = S.G[i], qi = scale * rqi;
-                SCg[ch * SC_FLOATS + i] = i < cn ? scale * expf(Gi) : 0.f;
-                if (i == 0) SCg[ch * SC_FLOATS + SC_GC] = expf(Gl);
-                uint4* prow = reinterpret_cast<uint4*>(Pg + (ch * 64 + i) * 64);
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    __align__(16) f16 e[8];
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        const int j = c8 * 8 + t;
+                    for (int j = 0; j < 64; ++j) {
                         float v = 0.f;
-                        if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
-                        e[t] = __float2half_rn(v);
+                        if (j < i && i < cn) v = bi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
+                        S.M[i][j] = v;
                     }
-                    prow[c8] = *reinterpret_cast<const uint4*>(e);
+                    SCg[ch * SC_FLOATS + 64 + i] = i < cn ? expf(Gl - Gi) : 0.f;
+                } else {
+                    const int i = tid - 64;
+                    const float Gi = S.G[i], qi = scale * rqi;
+                    SCg[ch * SC_FLOATS + i] = i < cn ? scale * expf(Gi) : 0.f;
+                    if (i == 0) SCg[ch * SC_FLOATS + SC_GC] = expf(Gl);
+                    uint4* prow = reinterpret_cast<uint4*>(Pg + (ch * 64 + i) * 64);
+#pragma unroll
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        __align__(16) f16 e[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int j = c8 * 8 + t;
+                            float v = 0.f;
+                            if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
+                            e[t] = __float2half_rn(v);
+                        }
+                        prow[c8] = *reinterpret_cast<const uint4*>(e);
+                    }
                 }
             }
             __syncthreads();
             tinv64_inplace(S.M, S.X, tid);
-            // ---- fp16 MMA operands T diag(b gamma) and T diag(b), 128B-swizzled ----------
+            // ---- fp16 MMA operands T diag(b gamma) and T diag(b), 128B-swizzled, written
+            //      over M once every thread holds its part of T -----------------------------
             {
                 const int i = tid >> 1, c0 = (tid & 1) * 32;
-                uint8_t* aw = reinterpret_cast<uint8_t*>(S.AW);
-                uint8_t* au = reinterpret_cast<uint8_t*>(S.AU);
+                float tv[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const int j = c0 + t;
+                    tv[t] = j < i ? S.M[i][j] : (j == i ? 1.f : 0.f);
+                }
+                __syncthreads();
+                uint8_t* aw = reinterpret_cast<uint8_t*>(&S.M[0][0]);
+                uint8_t* au = aw + 8192;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     __align__(16) f16 w8[8], u8[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
                         const int j = c0 + cc * 8 + t;
-                        const float tij = j < i ? S.M[i][j] : (j == i ? 1.f : 0.f);
-                        w8[t] = __float2half_rn(tij * S.bgr[j]);
-                        u8[t] = __float2half_rn(tij * S.bt[j]);
+                        w8[t] = __float2half_rn(tv[cc * 8 + t] * S.bgr[j]);
+                        u8[t] = __float2half_rn(tv[cc * 8 + t] * S.bt[j]);
                     }
                     const uint32_t off = tc::sw128_off(i, c0 + cc * 8);
                     *reinterpret_cast<uint4*>(aw + off) = *reinterpret_cast<const uint4*>(w8);
@@ -524,59 +558,53 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc::tc_fence_before();
             __syncthreads();
             // ---- W^T = K_hat^T AW^T and (V sv)^T AU^T (fp16, M=128, N=64, K=64 tokens) ----
+            const uint32_t kb = tc::smem_u32(kq), vb = kb + 8192;
+            const uint32_t awb = tc::smem_u32(&S.M[0][0]), aub = awb + 8192;
+            constexpr uint32_t idx = tc::idesc_f16(128, 64, 1, 0);
             if (tid == 0) {
                 tc::tc_fence_after();
-                const uint32_t kb = tc::smem_u32(kq), vb = kb + 8192;
-                const uint32_t awb = tc::smem_u32(S.AW), aub = tc::smem_u32(S.AU);
-                constexpr uint32_t idx = tc::idesc_f16(128, 64, 1, 0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tDW, tc::desc_sw128(kb + kk * 2048, 16384, 1024),
+                    tc::mma_bf16(tW, tc::desc_sw128(kb + kk * 2048, 16384, 1024),
                                  tc::desc_sw128(awb + kk * 32, 16, 1024), idx, kk > 0);
+                if (last) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tDU, tc::desc_sw128(vb + kk * 2048, 16384, 1024),
-                                 tc::desc_sw128(aub + kk * 32, 16, 1024), idx, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(tG, tc::desc_sw128(vb + kk * 2048, 16384, 1024),
+                                     tc::desc_sw128(aub + kk * 32, 16, 1024), idx, kk > 0);
+                }
                 tc::mma_commit(&S.bar_mma);
             }
-            ok = tc::mbar_wait(&S.bar_mma, (gi + 1) & 1);
+            ok = tc::mbar_wait(&S.bar_mma, mma_phase);
+            mma_phase ^= 1;
             if (__syncthreads_or(!ok)) goto abort;
             tc::tc_fence_after();
-            if (tid == 0 && gi + 1 < G) {   // the V rows are free again: next head's V
-                tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
-                tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, h + 1, si);
-                tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, h + 1, si);
-            }
-            // ---- epilogue: lane t of D_W / D_U is column t of W / U; stage the tiles in
-            //      shared memory, then copy each out as one contiguous 16 KB block ----------
-            {
-                f16* stw = S.AW;                                 // [64][128] fp16 (AW..AU)
-                f16* stu = reinterpret_cast<f16*>(&S.M[0][0]);   // [64][128] fp16
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    float w[32];
-                    tc::tmem_ld32(tDW + lane_base + part * 32, w);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) stw[(part * 32 + i) * D + tid] = __float2half_rn(w[i]);
-                    tc::tmem_ld32(tDU + lane_base + part * 32, w);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) stu[(part * 32 + i) * D + tid] = __float2half_rn(w[i]);
-                }
+            // ---- epilogue: lane t of D_W / D_U is column t of W / U -----------------------
+            store_tile_from_tmem(Wg + ch * 64 * D, tW + lane_base, tid);
+            if (!last) {   // U^T into the W^T columns once they are read
                 tc::tc_fence_before();
                 __syncthreads();
-                const uint4* sw4 = reinterpret_cast<const uint4*>(stw);
-                const uint4* su4 = reinterpret_cast<const uint4*>(stu);
-                uint4* gw4 = reinterpret_cast<uint4*>(Wg + ch * 64 * D);
-                uint4* gu4 = reinterpret_cast<uint4*>(Ug + ch * 64 * D);
+                if (tid == 0) {
+                    tc::tc_fence_after();
 #pragma unroll
-                for (int e = tid; e < 64 * D / 8; e += 128) {
-                    gw4[e] = sw4[e];
-                    gu4[e] = su4[e];
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(tW, tc::desc_sw128(vb + kk * 2048, 16384, 1024),
+                                     tc::desc_sw128(aub + kk * 32, 16, 1024), idx, kk > 0);
+                    tc::mma_commit(&S.bar_mma);
+                }
+                ok = tc::mbar_wait(&S.bar_mma, mma_phase);
+                mma_phase ^= 1;
+                if (__syncthreads_or(!ok)) goto abort;
+                tc::tc_fence_after();
+                if (tid == 0) {   // the V rows are free again: next head's V
+                    tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+                    tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, h + 1, si);
+                    tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, h + 1, si);
                 }
             }
-            __syncthreads();
+            store_tile_from_tmem(Ug + ch * 64 * D, (last ? tG : tW) + lane_base, tid);
+            tc::tc_fence_before();
+            __syncthreads();   // TMEM reads done; M (the operands) free for the next head
         }
     }
     tc::tc_fence_before();
@@ -1044,6 +1072,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
         if (G == 1) {
             e = cudaFuncSetAttribute(chunk_prep_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)kPrepSmemBytes);
+            if (e == cudaSuccess)   // four CTAs per SM need the largest shared-memory carveout
+                e = cudaFuncSetAttribute(chunk_prep_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return e;
             chunk_prep_kernel<1><<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T,
                                                                  a.n_seqs, a.HV, a.scale, a.l2norm, a.HK, W, U, P,
@@ -1051,6 +1082,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
         } else {
             e = cudaFuncSetAttribute(chunk_prep_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)kPrepSmemBytes);
+            if (e == cudaSuccess)   // four CTAs per SM need the largest shared-memory carveout
+                e = cudaFuncSetAttribute(chunk_prep_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return e;
             chunk_prep_kernel<2><<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T,
                                                                  a.n_seqs, a.HV, a.scale, a.l2norm, a.HK, W, U, P,
