@@ -676,8 +676,9 @@ __device__ __forceinline__ void store_op_row(f16* op, int k, const float* v, flo
 //   c: [0; P] Delta      (M=128, 4 MMAs)  -> D_c[c & 1]  rows 64-127 P Delta
 // Epilogue threads 0-63 turn D_a rows into Delta, Delta~; all 128 update the state rows
 // from D_b; threads 64-127 write the output rows of chunk c while chunk c+1's MMAs run.
-// The two sides meet only through mbarriers (h0_ready, d_ready: 128 arrivals each; the
-// output threads arrive on d_ready as soon as they have read the chunk's scalars, then
+// The two sides meet only through mbarriers (h0_ready, d_ready: one arrival per epilogue
+// warp, after its threads' shared-memory writes and proxy fences; the output warps
+// arrive on d_ready as soon as they have read the chunk's scalars, then
 // write the previous chunk's output rows while Delta and the state MMA proceed; the
 // stage is released only after every thread's reads of it).
 __global__ void __launch_bounds__(kCarryThreads, 1)
@@ -714,8 +715,8 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         tc::mbar_init(&S.bar_a, 1);
         tc::mbar_init(&S.bar_b, 1);
         tc::mbar_init(&S.bar_o, 1);
-        tc::mbar_init(&S.h0_ready, 128);
-        tc::mbar_init(&S.d_ready, 128);
+        tc::mbar_init(&S.h0_ready, 4);   // one arrival per epilogue warp
+        tc::mbar_init(&S.d_ready, 4);
         tc::fence_mbar_init();
         S.abort = 0;
     }
@@ -827,7 +828,8 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         const float sc = 1.f / inv_sc;
         store_op_row(S.H0[0], t, Hr, sc);
         tc::fence_async_smem();
-        tc::mbar_arrive(&S.h0_ready);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&S.h0_ready);
         bool ok = true;
         float a_prev = 0.f;
         int cn_prev = 0;
@@ -863,12 +865,14 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 store_op_row(S.Dt, t, dv, dr * sc);
                 tc::fence_async_smem();
                 tc::tc_fence_before();
-                tc::mbar_arrive(&S.d_ready);
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&S.d_ready);
             } else {
                 // ---- output rows of the previous chunk (threads 64-127), under this chunk's
                 //      Delta epilogue and state MMA -------------------------------------------
                 const float a_cur = B.SC[t - 64];
-                tc::mbar_arrive(&S.d_ready);   // the stage's scalars are read
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&S.d_ready);   // the stage's scalars are read
                 if (c > 0) {
                     ok = tc::mbar_wait(&S.bar_o, (c - 1) & 1) && ok;
                     tc::tc_fence_after();
@@ -903,7 +907,8 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
             store_op_row(S.H0[(c + 1) & 1], t, Hr, sc);
             tc::fence_async_smem();
             tc::tc_fence_before();
-            tc::mbar_arrive(&S.h0_ready);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&S.h0_ready);
             if (S.abort) ok = false;
         }
         if (ok && nch > 0 && warp >= 2) {   // output rows of the last chunk
