@@ -48,6 +48,7 @@ _SIGS = {
     "gdn_chunk_prefill_status": ([_vp, _vp, ctypes.POINTER(_i32)], ctypes.c_int),
     "gdn_decode_step": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                          _f32, _i32, _vp, _vp], ctypes.c_int),
+    "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
 }
 
 _LIB = None
@@ -203,3 +204,12 @@ def gdn_decode_step(q, k, v, g, beta, state, scale: float = 1.0, qk_l2norm: bool
                                _ptr(o), _stream())
     _check(st, "gdn_decode_step")
     return o
+
+
+def gdn_decode_status() -> int:
+    """Synchronise the device, return its decode error word and clear it."""
+    word = _i32(0)
+    st = lib().gdn_decode_status(ctypes.byref(word))
+    if st not in (0, 8):
+        _check(st, "gdn_decode_status")
+    return int(word.value)

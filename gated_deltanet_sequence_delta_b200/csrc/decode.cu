@@ -13,9 +13,23 @@
 // Dv/32 contiguous columns, so every warp load/store is a contiguous 8 x 512-byte
 // (Dv = 128) burst of 128-bit accesses.  The Dk reduction is a per-thread sum over
 // 8 rows, then a cross-warp sum through shared memory.
+//
+// For Dk = Dv = 128 a persistent variant streams the slices through shared memory: one CTA
+// per SM, a producer warp keeps a ring of three slices in flight with bulk copies
+// (64 KB of state plus the q, k, v rows per slice), sixteen warps update each slice in
+// shared memory with the same arithmetic and mapping, and one thread writes it back with
+// a bulk store.  HBM then sees a steady stream of loads and stores instead of the gaps
+// between short-lived CTAs.
+#include <mutex>
+
 #include "gdn_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace gdn {
+
+// set (to GDN_DEVERR_TIMEOUT) by a staged decode launch whose bounded wait expired
+__device__ int32_t g_decode_error = 0;
+
 namespace {
 
 template <int CPL>
@@ -140,6 +154,195 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
     }
 }
 
+// ---- persistent, shared-memory staged variant (Dk = Dv = 128) --------------------------
+constexpr int kSD = 128;                   // Dk = Dv of this variant
+constexpr int kSStages = 3;
+constexpr int kSWarps = 16;                // compute warps: rows 8w .. 8w+7 each
+constexpr int kSThreads = kSWarps * 32 + 32;   // + producer warp
+struct StagedSlot {
+    float H[kSD * kSD];                    // the state slice, row-major as in global memory
+    __align__(16) uint8_t q[kSD * 4], k[kSD * 4], v[kSD * 4];   // raw rows (bf16 or fp32)
+};
+struct StagedSmem {
+    StagedSlot st[kSStages];
+    float red_u[kSWarps][kSD], red_q[kSWarps][kSD];
+    float delta[kSD];
+    float dot[4];
+    uint64_t full[kSStages], empty[kSStages];
+};
+constexpr size_t kStagedSmemBytes = sizeof(StagedSmem) + 128;
+
+template <typename IO>
+__device__ __forceinline__ float ld_raw(const uint8_t* p, int i) {
+    return load_elem(reinterpret_cast<const IO*>(p), i);
+}
+
+template <typename IO>
+__global__ void __launch_bounds__(kSThreads, 1)
+decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
+                     const float* __restrict__ g, const float* __restrict__ beta,
+                     float* __restrict__ state, int n_items, int HK, int HV, float scale, int l2norm,
+                     IO* __restrict__ o) {
+    constexpr int CPL = kSD / 32;   // 4 columns per lane
+    constexpr uint32_t kRowBytes = kSD * sizeof(IO);
+    constexpr uint32_t kTx = kSD * kSD * 4 + 3 * kRowBytes;
+    extern __shared__ uint8_t smem_raw[];
+    StagedSmem& S = *reinterpret_cast<StagedSmem*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x;
+    const int n_mine = blockIdx.x < n_items ? (n_items - 1 - blockIdx.x) / G + 1 : 0;
+    if (tid == 0) {
+        for (int i = 0; i < kSStages; ++i) {
+            tc::mbar_init(&S.full[i], 1);
+            tc::mbar_init(&S.empty[i], 1);
+        }
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kSWarps) {
+        // ---------------- producer ----------------------------------------------------
+        if (lane == 0) {
+            for (int i = 0; i < n_mine; ++i) {
+                const int st = i % kSStages, r = i / kSStages;
+                if (r > 0 && !tc::mbar_wait(&S.empty[st], (r - 1) & 1)) {
+                    atomicExch(&g_decode_error, GDN_DEVERR_TIMEOUT);
+                    break;
+                }
+                const int bh = blockIdx.x + i * G;
+                const int b = bh / HV, h = bh - b * HV, hk = h / (HV / HK);
+                StagedSlot& B = S.st[st];
+                tc::mbar_expect_tx(&S.full[st], kTx);
+                const float* src = state + (size_t)bh * kSD * kSD;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) tc::bulk_load(B.H + p * 4096, src + p * 4096, 16384, &S.full[st]);
+                tc::bulk_load(B.q, q + ((size_t)b * HK + hk) * kSD, kRowBytes, &S.full[st]);
+                tc::bulk_load(B.k, k + ((size_t)b * HK + hk) * kSD, kRowBytes, &S.full[st]);
+                tc::bulk_load(B.v, v + (size_t)bh * kSD, kRowBytes, &S.full[st]);
+            }
+        }
+        return;   // the producer takes part in no later barrier
+    }
+
+    // ---------------- 512 compute threads (named barrier 1) ------------------------------
+    for (int i = 0; i < n_mine; ++i) {
+        const int st = i % kSStages, r = i / kSStages;
+        const int bh = blockIdx.x + i * G;
+        StagedSlot& B = S.st[st];
+        const float alpha = expf(g[bh]);   // issued before the wait
+        const float bt = beta[bh];
+        const bool ok = tc::mbar_wait(&S.full[st], r & 1);
+        if (tc::named_bar_any(1, kSWarps * 32, !ok)) {   // uniform decision to stop
+            if (tid == 0) atomicExch(&g_decode_error, GDN_DEVERR_TIMEOUT);
+            break;
+        }
+        // norms and k.q (warps 0-2), partial column sums over this warp's 8 rows
+        if (warp < 3) {
+            float acc = 0.f;
+            for (int e = lane; e < kSD; e += 32) {
+                const float x = warp == 1 ? ld_raw<IO>(B.k, e) : ld_raw<IO>(B.q, e);
+                const float y = warp == 0 ? ld_raw<IO>(B.q, e) : ld_raw<IO>(B.k, e);
+                acc += x * y;   // warp 0: q.q, warp 1: k.k, warp 2: q.k
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) S.dot[warp] = acc;
+        }
+        float4 hv[8];
+        float pu[CPL] = {}, pq[CPL] = {};
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            const int row = warp * 8 + rr;
+            hv[rr] = *reinterpret_cast<const float4*>(B.H + row * kSD + lane * CPL);
+            const float kr = ld_raw<IO>(B.k, row), qr = ld_raw<IO>(B.q, row);
+            const float hf[4] = {hv[rr].x, hv[rr].y, hv[rr].z, hv[rr].w};
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                pu[c] = fmaf(kr, hf[c], pu[c]);
+                pq[c] = fmaf(qr, hf[c], pq[c]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            S.red_u[warp][lane * CPL + c] = pu[c];
+            S.red_q[warp][lane * CPL + c] = pq[c];
+        }
+        tc::named_bar(1, kSWarps * 32);
+        const float rq = l2_inv(S.dot[0], l2norm);
+        const float rk = l2_inv(S.dot[1], l2norm);
+        const float kq = S.dot[2] * rq * rk;
+        if (tid < kSD) {   // column sums, delta and the output
+            const int j = tid;
+            float su = 0.f, sq = 0.f;
+#pragma unroll
+            for (int w = 0; w < kSWarps; ++w) {
+                su += S.red_u[w][j];
+                sq += S.red_q[w][j];
+            }
+            const float delta = bt * (ld_raw<IO>(B.v, j) - alpha * su * rk);
+            store_elem(o, (int64_t)bh * kSD + j, scale * (alpha * (sq * rq) + delta * kq));
+            S.delta[j] = delta;
+        }
+        tc::named_bar(1, kSWarps * 32);
+        // H' = alpha H + k_hat delta^T, written back in place
+        const float4 dl = *reinterpret_cast<const float4*>(&S.delta[lane * CPL]);
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            const int row = warp * 8 + rr;
+            const float kr = ld_raw<IO>(B.k, row) * rk;
+            float4 x = hv[rr];
+            x.x = fmaf(alpha, x.x, kr * dl.x);
+            x.y = fmaf(alpha, x.y, kr * dl.y);
+            x.z = fmaf(alpha, x.z, kr * dl.z);
+            x.w = fmaf(alpha, x.w, kr * dl.w);
+            *reinterpret_cast<float4*>(B.H + row * kSD + lane * CPL) = x;
+        }
+        tc::fence_async_smem();
+        tc::named_bar(1, kSWarps * 32);
+        if (tid == 0) {
+            float* dst = state + (size_t)bh * kSD * kSD;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) tc::bulk_store(dst + p * 4096, B.H + p * 4096, 16384);
+            tc::bulk_commit();
+            tc::bulk_wait_read<1>();   // the previous slice's store has read its slot
+            if (i > 0) tc::mbar_arrive(&S.empty[(i - 1) % kSStages]);
+        }
+    }
+    if (tid == 0) tc::bulk_wait<0>();   // every store complete before the CTA exits
+}
+
+int staged_grid() {
+    static std::mutex mu;
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!sms[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        sms[dev] = n;
+    }
+    return sms[dev];
+}
+
+template <typename IO>
+cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, float* state, int B, int HK, int HV, float scale,
+                                 int l2norm, void* o, cudaStream_t s) {
+    const int n_items = B * HV;
+    const int sms = staged_grid();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kStagedSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int grid = n_items < sms ? n_items : sms;
+    decode_staged_kernel<IO><<<grid, kSThreads, kStagedSmemBytes, s>>>(
+        (const IO*)q, (const IO*)k, (const IO*)v, g, beta, state, n_items, HK, HV, scale, l2norm, (IO*)o);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launch();
+    return e;
+}
+
 template <int DK, int DV, typename IO>
 cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* g,
                             const float* beta, float* state, int B, int HK, int HV, float scale,
@@ -159,18 +362,29 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16
                           int HV, int Dk, int Dv, float scale, int l2norm, void* o,
                           cudaStream_t s) {
     if (B == 0) return cudaSuccess;
+    if (Dk == kSD && Dv == kSD)   // the API guarantees 16-byte aligned pointers
+        return bf16 ? launch_decode_staged<__nv_bfloat16>(q, k, v, g, beta, state, B, HK, HV, scale, l2norm, o, s)
+                    : launch_decode_staged<float>(q, k, v, g, beta, state, B, HK, HV, scale, l2norm, o, s);
 #define GDN_DECODE_CASE(DK_, DV_)                                                                \
     if (Dk == DK_ && Dv == DV_)                                                                  \
         return bf16 ? launch_decode_t<DK_, DV_, __nv_bfloat16>(q, k, v, g, beta, state, B, HK,   \
                                                                HV, scale, l2norm, o, s)          \
                     : launch_decode_t<DK_, DV_, float>(q, k, v, g, beta, state, B, HK, HV,       \
                                                        scale, l2norm, o, s);
-    GDN_DECODE_CASE(128, 128)
     GDN_DECODE_CASE(128, 64)
     GDN_DECODE_CASE(64, 128)
     GDN_DECODE_CASE(64, 64)
 #undef GDN_DECODE_CASE
     return cudaErrorInvalidValue;
+}
+
+cudaError_t read_decode_error(int32_t* out, bool reset) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_decode_error, sizeof(int32_t));
+    if (e == cudaSuccess && reset && *out != 0) {
+        const int32_t zero = 0;
+        e = cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(int32_t));
+    }
+    return e;
 }
 
 }  // namespace gdn

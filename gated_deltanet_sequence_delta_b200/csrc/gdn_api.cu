@@ -202,4 +202,15 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtyp
                                           Dk, Dv, scale, qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
 }
 
+gdn_status gdn_decode_status(int32_t* device_error) {
+    if (!device_error) return GDN_ERR_NULL;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e);
+    int32_t word = 0;
+    e = gdn::read_decode_error(&word, true);
+    if (e != cudaSuccess) return cuda_status(e);
+    *device_error = word;
+    return word ? GDN_ERR_DEVICE : GDN_OK;
+}
+
 }  // extern "C"

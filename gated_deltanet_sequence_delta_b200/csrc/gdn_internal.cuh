@@ -51,6 +51,9 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16
                           int HV, int Dk, int Dv, float scale, int l2norm, void* o,
                           cudaStream_t s);
 
+// Read (and on request clear) the device word a staged decode launch sets on a timeout.
+cudaError_t read_decode_error(int32_t* out, bool reset);
+
 struct PrefillArgs {
     const void* q;
     const void* k;

@@ -200,12 +200,24 @@ GDN_API gdn_status gdn_chunk_prefill_static_ws(const void* q, const void* k, con
  *   o      [B, HV, Dv] io_dtype                            (written; o = scale * S_t q_t
  *                                                           with the updated state)
  * B may be 0 (nothing launched).
+ * For Dk = Dv = 128 the step runs as a persistent kernel whose waits are bounded; if one
+ * expires (no such case is known) the launch stops early and records
+ * GDN_DEVERR_TIMEOUT, which gdn_decode_status reports.
  * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, ALIAS, CUDA.
  */
 GDN_API gdn_status gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
                            const float* g, const float* beta, float* state,
                            int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
                            float scale, int32_t qk_l2norm, void* o, void* stream);
+
+/*
+ * gdn_decode_status -- synchronises the current device and writes its decode error
+ * word (GDN_DEVERR_NONE or GDN_DEVERR_TIMEOUT, shared by every decode launch on that
+ * device) into *device_error, then clears it.  This is library bookkeeping with no
+ * counterpart in the method.  Returns OK if the word was 0, DEVICE if not, NULL for a
+ * NULL argument, CUDA on a CUDA error.
+ */
+GDN_API gdn_status gdn_decode_status(int32_t* device_error);
 
 #ifdef __cplusplus
 }

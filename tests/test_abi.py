@@ -105,6 +105,10 @@ def test_decode_validation(L):
     assert call(a7=0) == 0                      # B = 0: nothing to do
 
 
+def test_decode_status_null(L):
+    assert L.gdn_decode_status(None) == 1
+
+
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(binding.GDNLibraryError):
         binding.lib(str(tmp_path / "nope.so"))

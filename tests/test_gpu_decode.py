@@ -60,8 +60,10 @@ def test_decode_small(io, D):
 
 def test_decode_workload_first_steps_all_heads():
     """B=64, H=32, d=128, bf16: the first 16 steps on every (sequence, head)."""
+    import gated_deltanet_sequence_delta_b200 as G
     setup = I.decode()
     _run_steps(setup, 16)
+    assert G.gdn_decode_status() == 0   # no bounded wait expired
 
 
 def test_decode_workload_all_steps_sampled():
@@ -71,6 +73,8 @@ def test_decode_workload_all_steps_sampled():
     rng = np.random.default_rng(123)
     pairs = sorted({(int(rng.integers(64)), int(rng.integers(32))) for _ in range(12)} | {(0, 0), (63, 31)})
     _run_steps(setup, I.DECODE_STEPS, sample=pairs, check_every=64)
+    import gated_deltanet_sequence_delta_b200 as G
+    assert G.gdn_decode_status() == 0
 
 
 def test_decode_no_write_no_decay_keeps_state():
