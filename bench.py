@@ -421,13 +421,31 @@ def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, 
     barrier()
     clocks.window(w0, time.time())
     dec_kernel_ms = max_over_ranks(k0.elapsed_time(k1) / n_dec)
+    # the step with the gates formed inside the kernel (one launch per step)
+    nf0 = G.kernel_launches()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    f0.record()
+    for i in range(n_dec):
+        dq, dk, dv, da, db = ring[i % len(ring)]
+        G.gdn_decode_step_gated(dq, dk, dv, da, db, dA, dbias, state, o=do)
+    f1.record()
+    barrier()
+    clocks.window(w0, time.time())
+    gated_launches = G.kernel_launches() - nf0
+    gated_ms = max_over_ranks(f0.elapsed_time(f1) / n_dec)
     dbytes = decode_bytes_per_step(ds.B, ds.HK, ds.HV, ds.Dk, ds.Dv)
     dgbs = dbytes / (dec_kernel_ms * 1e-3) / 1e9
+    ggbs = dbytes / (gated_ms * 1e-3) / 1e9
     return {"workload": "decode: B=64 HK=HV=32 Dk=Dv=128 bf16 q/k/v, fp32 state 128 MiB, "
                         f"{n_dec} consecutive steps (gates + step), inputs cycled from 8 resident steps",
             "ms_per_step": dec_ms, "steps_per_s": world * 1e3 / dec_ms,
             "tokens_per_s": world * ds.B * 1e3 / dec_ms,
             "gpu_launches": dec_launches,
+            "gated_step": {"what": "gdn_decode_step_gated: gates formed in the decode kernel, one launch per step",
+                           "ms_per_step": gated_ms, "steps_per_s": world * 1e3 / gated_ms,
+                           "achieved_gbs": ggbs, "frac": ggbs / P["hbm_gbs"], "gpu_launches": gated_launches},
             "roofline": {"bound": "hbm", "achieved": dgbs, "peak": P["hbm_gbs"], "unit": "GB/s",
                          "frac": dgbs / P["hbm_gbs"],
                          "traffic": _traffic().get("decode_bytes_per_launch"),

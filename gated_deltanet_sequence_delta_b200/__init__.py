@@ -5,7 +5,8 @@ is its thin binding.  Names are re-exported lazily so that ``inputs`` (the
 seeded workload generator) can be imported without loading torch or the
 library.
 """
-_BINDING = ("gdn_gates", "gdn_chunk_prefill", "gdn_chunk_prefill_status", "gdn_decode_step", "gdn_decode_status",
+_BINDING = ("gdn_gates", "gdn_chunk_prefill", "gdn_chunk_prefill_status", "gdn_decode_step", "gdn_decode_step_gated",
+            "gdn_decode_status",
             "GDNError", "GDNLibraryError", "prefill_workspace_bytes", "kernel_launches")
 
 __all__ = list(_BINDING)

@@ -49,6 +49,8 @@ _SIGS = {
     "gdn_decode_step": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                          _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_decode_step_gated": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32,
+                               _i32, _i32, _i32, _f32, _i32, _vp, _vp], ctypes.c_int),
 }
 
 _LIB = None
@@ -203,6 +205,29 @@ def gdn_decode_step(q, k, v, g, beta, state, scale: float = 1.0, qk_l2norm: bool
                                _ptr(state), B, HK, HV, Dk, Dv, float(scale), int(bool(qk_l2norm)),
                                _ptr(o), _stream())
     _check(st, "gdn_decode_step")
+    return o
+
+
+def gdn_decode_step_gated(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0, qk_l2norm: bool = True,
+                          o=None):
+    """gdn_decode_step with the gates formed in the kernel: a, b [B, HV] (fp32 or bf16),
+    A_log, dt_bias [HV] fp32 instead of g, beta.  Returns o [B, HV, Dv]."""
+    B, HK, Dk = q.shape
+    HV, Dv = v.shape[-2:]
+    if k.shape != q.shape or v.shape[0] != B or a.shape != (B, HV) or b.shape != (B, HV):
+        raise ValueError("inconsistent decode shapes")
+    if a.dtype != b.dtype or A_log.shape != (HV,) or dt_bias.shape != (HV,):
+        raise ValueError("a, b must share a dtype; A_log, dt_bias must be [HV]")
+    if A_log.dtype != torch.float32 or dt_bias.dtype != torch.float32:
+        raise ValueError("A_log and dt_bias must be fp32")
+    if state.shape != (B, HV, Dk, Dv) or state.dtype != torch.float32:
+        raise ValueError("state must be fp32 [B, HV, Dk, Dv]")
+    if o is None:
+        o = torch.empty((B, HV, Dv), dtype=q.dtype, device=q.device)
+    st = lib().gdn_decode_step_gated(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(a), _ptr(b), _dtype_code(a),
+                                     _ptr(A_log), _ptr(dt_bias), _ptr(state), B, HK, HV, Dk, Dv, float(scale),
+                                     int(bool(qk_l2norm)), _ptr(o), _stream())
+    _check(st, "gdn_decode_step_gated")
     return o
 
 

@@ -52,8 +52,7 @@ struct VecF<2> {
 template <int DK, int DV, typename IO>
 __global__ void __launch_bounds__(DK * 4, (DK == 128 ? 2 : 4))
 decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
-              const float* __restrict__ g, const float* __restrict__ beta,
-              float* __restrict__ state, int HK, int HV, float scale, int l2norm,
+              const DecodeGates gates, float* __restrict__ state, int HK, int HV, float scale, int l2norm,
               IO* __restrict__ o) {
     constexpr int NW = DK / 8;      // warps; 8 state rows each
     constexpr int CPL = DV / 32;    // state columns per lane
@@ -118,8 +117,9 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
     const float rq = l2_inv(s_dot[0], l2norm);
     const float rk = l2_inv(s_dot[1], l2norm);
     const float kq = s_dot[2] * rq * rk;
-    const float alpha = expf(g[bh]);
-    const float bt = beta[bh];
+    float gv, bt;
+    decode_gates(gates, bh, h, gv, bt);
+    const float alpha = expf(gv);
 
     // 4. column sums, delta and the output (threads 0 .. DV-1); delta -> shared
     float* s_delta = &s_red_u[0][0];   // row 0 reused after its value is consumed
@@ -180,9 +180,8 @@ __device__ __forceinline__ float ld_raw(const uint8_t* p, int i) {
 template <typename IO>
 __global__ void __launch_bounds__(kSThreads, 1)
 decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
-                     const float* __restrict__ g, const float* __restrict__ beta,
-                     float* __restrict__ state, int n_items, int HK, int HV, float scale, int l2norm,
-                     IO* __restrict__ o) {
+                     const DecodeGates gates, float* __restrict__ state, int n_items, int HK, int HV,
+                     float scale, int l2norm, IO* __restrict__ o) {
     constexpr int CPL = kSD / 32;   // 4 columns per lane
     constexpr uint32_t kRowBytes = kSD * sizeof(IO);
     constexpr uint32_t kTx = kSD * kSD * 4 + 3 * kRowBytes;
@@ -230,8 +229,9 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
         const int st = i % kSStages, r = i / kSStages;
         const int bh = blockIdx.x + i * G;
         StagedSlot& B = S.st[st];
-        const float alpha = expf(g[bh]);   // issued before the wait
-        const float bt = beta[bh];
+        float gv, bt;
+        decode_gates(gates, bh, bh % HV, gv, bt);   // issued before the wait
+        const float alpha = expf(gv);
         const bool ok = tc::mbar_wait(&S.full[st], r & 1);
         if (tc::named_bar_any(1, kSWarps * 32, !ok)) {   // uniform decision to stop
             if (tid == 0) atomicExch(&g_decode_error, GDN_DEVERR_TIMEOUT);
@@ -326,9 +326,9 @@ int staged_grid() {
 }
 
 template <typename IO>
-cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, const float* g,
-                                 const float* beta, float* state, int B, int HK, int HV, float scale,
-                                 int l2norm, void* o, cudaStream_t s) {
+cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, const DecodeGates& gates,
+                                 float* state, int B, int HK, int HV, float scale, int l2norm, void* o,
+                                 cudaStream_t s) {
     const int n_items = B * HV;
     const int sms = staged_grid();
     if (sms <= 0) return cudaErrorInvalidDevice;
@@ -337,19 +337,19 @@ cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, co
     if (e != cudaSuccess) return e;
     const int grid = n_items < sms ? n_items : sms;
     decode_staged_kernel<IO><<<grid, kSThreads, kStagedSmemBytes, s>>>(
-        (const IO*)q, (const IO*)k, (const IO*)v, g, beta, state, n_items, HK, HV, scale, l2norm, (IO*)o);
+        (const IO*)q, (const IO*)k, (const IO*)v, gates, state, n_items, HK, HV, scale, l2norm, (IO*)o);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
 }
 
 template <int DK, int DV, typename IO>
-cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* g,
-                            const float* beta, float* state, int B, int HK, int HV, float scale,
-                            int l2norm, void* o, cudaStream_t s) {
+cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const DecodeGates& gates,
+                            float* state, int B, int HK, int HV, float scale, int l2norm, void* o,
+                            cudaStream_t s) {
     const unsigned blocks = (unsigned)B * (unsigned)HV;
     decode_kernel<DK, DV, IO><<<blocks, DK * 4, 0, s>>>(
-        (const IO*)q, (const IO*)k, (const IO*)v, g, beta, state, HK, HV, scale, l2norm, (IO*)o);
+        (const IO*)q, (const IO*)k, (const IO*)v, gates, state, HK, HV, scale, l2norm, (IO*)o);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
@@ -357,20 +357,18 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const f
 
 }  // namespace
 
-cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16,
-                          const float* g, const float* beta, float* state, int B, int HK,
-                          int HV, int Dk, int Dv, float scale, int l2norm, void* o,
+cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16, const DecodeGates& gates,
+                          float* state, int B, int HK, int HV, int Dk, int Dv, float scale, int l2norm, void* o,
                           cudaStream_t s) {
     if (B == 0) return cudaSuccess;
     if (Dk == kSD && Dv == kSD)   // the API guarantees 16-byte aligned pointers
-        return bf16 ? launch_decode_staged<__nv_bfloat16>(q, k, v, g, beta, state, B, HK, HV, scale, l2norm, o, s)
-                    : launch_decode_staged<float>(q, k, v, g, beta, state, B, HK, HV, scale, l2norm, o, s);
-#define GDN_DECODE_CASE(DK_, DV_)                                                                \
-    if (Dk == DK_ && Dv == DV_)                                                                  \
-        return bf16 ? launch_decode_t<DK_, DV_, __nv_bfloat16>(q, k, v, g, beta, state, B, HK,   \
-                                                               HV, scale, l2norm, o, s)          \
-                    : launch_decode_t<DK_, DV_, float>(q, k, v, g, beta, state, B, HK, HV,       \
-                                                       scale, l2norm, o, s);
+        return bf16 ? launch_decode_staged<__nv_bfloat16>(q, k, v, gates, state, B, HK, HV, scale, l2norm, o, s)
+                    : launch_decode_staged<float>(q, k, v, gates, state, B, HK, HV, scale, l2norm, o, s);
+#define GDN_DECODE_CASE(DK_, DV_)                                                                  \
+    if (Dk == DK_ && Dv == DV_)                                                                    \
+        return bf16 ? launch_decode_t<DK_, DV_, __nv_bfloat16>(q, k, v, gates, state, B, HK, HV, scale, \
+                                                               l2norm, o, s)                       \
+                    : launch_decode_t<DK_, DV_, float>(q, k, v, gates, state, B, HK, HV, scale, l2norm, o, s);
     GDN_DECODE_CASE(128, 64)
     GDN_DECODE_CASE(64, 128)
     GDN_DECODE_CASE(64, 64)

@@ -15,9 +15,10 @@ __global__ void __launch_bounds__(256) gates_kernel(const T* __restrict__ a, con
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         const int h = (int)(i % HV);
-        const float x = load_elem(a, i) + __ldg(dt_bias + h);
-        g[i] = -expf(__ldg(A_log + h)) * softplus_f(x);
-        beta[i] = 1.0f / (1.0f + expf(-load_elem(b, i)));
+        float gv, bv;
+        gate_pair(load_elem(a, i), load_elem(b, i), __ldg(A_log + h), __ldg(dt_bias + h), gv, bv);
+        g[i] = gv;
+        beta[i] = bv;
     }
 }
 

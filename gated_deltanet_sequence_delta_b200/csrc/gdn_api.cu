@@ -198,8 +198,35 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtyp
         for (Range in : {rq, rk, rv, rg, rb})
             if (overlap(out, in)) return GDN_ERR_ALIAS;
     if (overlap(rs, ro)) return GDN_ERR_ALIAS;
-    return cuda_status(gdn::launch_decode(q, k, v, io_dtype == GDN_BF16, g, beta, state, B, HK, HV,
-                                          Dk, Dv, scale, qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
+    const gdn::DecodeGates gates{g, beta, nullptr, nullptr, false, nullptr, nullptr};
+    return cuda_status(gdn::launch_decode(q, k, v, io_dtype == GDN_BF16, gates, state, B, HK, HV, Dk, Dv, scale,
+                                          qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
+}
+
+gdn_status gdn_decode_step_gated(const void* q, const void* k, const void* v, gdn_dtype io_dtype, const void* a,
+                                 const void* b, gdn_dtype ab_dtype, const float* A_log, const float* dt_bias,
+                                 float* state, int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                                 float scale, int32_t qk_l2norm, void* o, void* stream) {
+    if (B < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || HV % HK != 0) return GDN_ERR_SHAPE;
+    if (!dtype_ok(io_dtype) || !dtype_ok(ab_dtype) || !head_dim_ok(Dk) || !head_dim_ok(Dv))
+        return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state || !o) return GDN_ERR_NULL;
+    const void* ptrs[] = {q, k, v, a, b, A_log, dt_bias, state, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t es = esize(io_dtype), eab = esize(ab_dtype);
+    const Range rq{q, (size_t)B * HK * Dk * es}, rk{k, (size_t)B * HK * Dk * es};
+    const Range rv{v, (size_t)B * HV * Dv * es}, ra{a, (size_t)B * HV * eab}, rb{b, (size_t)B * HV * eab};
+    const Range rA{A_log, (size_t)HV * 4}, rd{dt_bias, (size_t)HV * 4};
+    const Range rs{state, (size_t)B * HV * Dk * Dv * 4}, ro{o, (size_t)B * HV * Dv * es};
+    for (Range out : {rs, ro})
+        for (Range in : {rq, rk, rv, ra, rb, rA, rd})
+            if (overlap(out, in)) return GDN_ERR_ALIAS;
+    if (overlap(rs, ro)) return GDN_ERR_ALIAS;
+    const gdn::DecodeGates gates{nullptr, nullptr, a, b, ab_dtype == GDN_BF16, A_log, dt_bias};
+    return cuda_status(gdn::launch_decode(q, k, v, io_dtype == GDN_BF16, gates, state, B, HK, HV, Dk, Dv, scale,
+                                          qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
 }
 
 gdn_status gdn_decode_status(int32_t* device_error) {

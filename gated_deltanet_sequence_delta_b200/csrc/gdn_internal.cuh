@@ -30,6 +30,14 @@ __device__ __forceinline__ float softplus_f(float x) {
     return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
 }
 
+// The gates ("Gated DeltaNet ... Qwen3-next" page, section 2.1) of one (token, value head):
+// g = -exp(A_log) * softplus(a + dt_bias), beta = sigmoid(b).  Every kernel that forms
+// gates calls this, so a fused gate prologue is bit-identical to gdn_gates.
+__device__ __forceinline__ void gate_pair(float a, float b, float A_log, float dt_bias, float& g, float& beta) {
+    g = -expf(A_log) * softplus_f(a + dt_bias);
+    beta = 1.0f / (1.0f + expf(-b));
+}
+
 // L2-normalisation factor 1 / sqrt(sum x^2 + 1e-6) (flag off: 1).
 __device__ __forceinline__ float l2_inv(float sumsq, int enabled) {
     return enabled ? 1.0f / sqrtf(sumsq + 1e-6f) : 1.0f;
@@ -46,9 +54,31 @@ cudaError_t launch_gates(const void* a, const void* b, bool ab_bf16, const float
                          const float* dt_bias, int64_t n_tokens, int HV, float* g, float* beta,
                          cudaStream_t s);
 
-cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16,
-                          const float* g, const float* beta, float* state, int B, int HK,
-                          int HV, int Dk, int Dv, float scale, int l2norm, void* o,
+// Where a decode step takes its gates from: g, beta [B, HV] as given, or (g == nullptr)
+// formed in the kernel from a, b [B, HV] (bf16 or fp32) and A_log, dt_bias [HV].
+struct DecodeGates {
+    const float* g;
+    const float* beta;
+    const void* a;
+    const void* b;
+    bool ab_bf16;
+    const float* A_log;
+    const float* dt_bias;
+};
+__device__ __forceinline__ void decode_gates(const DecodeGates& G, int bh, int h, float& g, float& beta) {
+    if (G.g) {
+        g = G.g[bh];
+        beta = G.beta[bh];
+    } else if (G.ab_bf16) {
+        gate_pair(load_elem((const __nv_bfloat16*)G.a, bh), load_elem((const __nv_bfloat16*)G.b, bh), G.A_log[h],
+                  G.dt_bias[h], g, beta);
+    } else {
+        gate_pair(((const float*)G.a)[bh], ((const float*)G.b)[bh], G.A_log[h], G.dt_bias[h], g, beta);
+    }
+}
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16, const DecodeGates& gates,
+                          float* state, int B, int HK, int HV, int Dk, int Dv, float scale, int l2norm, void* o,
                           cudaStream_t s);
 
 // Read (and on request clear) the device word a staged decode launch sets on a timeout.

@@ -211,6 +211,23 @@ GDN_API gdn_status gdn_decode_step(const void* q, const void* k, const void* v, 
                            float scale, int32_t qk_l2norm, void* o, void* stream);
 
 /*
+ * gdn_decode_step_gated -- the same step with the gate prologue fused in: g and beta are
+ * formed inside the kernel from the raw gate inputs with the formula of gdn_gates
+ * ("Gated DeltaNet ... Qwen3-next" page, section 2.1), bit for bit as gdn_gates would
+ * write them, instead of being read from memory.  Saves the separate gates launch and its
+ * round trip through HBM on every decode step.
+ *   a, b     [B, HV] ab_dtype (fp32 or bf16)                 (read)
+ *   A_log, dt_bias [HV] fp32                                  (read)
+ *   other arguments as gdn_decode_step.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, ALIAS (state or o over any input), CUDA.
+ */
+GDN_API gdn_status gdn_decode_step_gated(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                           const void* a, const void* b, gdn_dtype ab_dtype,
+                           const float* A_log, const float* dt_bias, float* state,
+                           int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                           float scale, int32_t qk_l2norm, void* o, void* stream);
+
+/*
  * gdn_decode_status -- synchronises the current device and writes its decode error
  * word (GDN_DEVERR_NONE or GDN_DEVERR_TIMEOUT, shared by every decode launch on that
  * device) into *device_error, then clears it.  This is library bookkeeping with no

@@ -105,6 +105,27 @@ def test_decode_validation(L):
     assert call(a7=0) == 0                      # B = 0: nothing to do
 
 
+def test_decode_gated_validation(L):
+    f = L.gdn_decode_step_gated
+    # q, k, v, io, a, b, ab, A_log, dt_bias, state, B, HK, HV, Dk, Dv, scale, l2, o, stream
+    base = [A, A + MB, A + 2 * MB, 1, A + 3 * MB, A + 4 * MB, 0, A + 5 * MB, A + 6 * MB, A + 16 * MB,
+            4, 2, 4, 128, 128, 1.0, 1, A + 8 * MB, None]
+    def call(**kw):
+        a = list(base)
+        for i, val in kw.items():
+            a[int(i[1:])] = val
+        return f(*a)
+    assert call(a4=None) == 1                   # a missing
+    assert call(a8=None) == 1                   # dt_bias missing
+    assert call(a12=3) == 2                     # HV % HK
+    assert call(a6=7) == 4                      # bad ab dtype
+    assert call(a13=32) == 4                    # head dim
+    assert call(a5=A + 4 * MB + 4) == 3         # b misaligned
+    assert call(a17=A + 3 * MB) == 5            # o over a
+    assert call(a9=A + 5 * MB) == 5             # state over A_log
+    assert call(a10=0) == 0                     # B = 0: nothing to do
+
+
 def test_decode_status_null(L):
     assert L.gdn_decode_status(None) == 1
 

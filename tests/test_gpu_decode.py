@@ -8,9 +8,10 @@ from harness import TOL, assert_close, to_dev, to_np
 pytestmark = pytest.mark.gpu
 
 
-def _run_steps(setup, n_steps, sample=None, check_every=1):
+def _run_steps(setup, n_steps, sample=None, check_every=1, fused_gates=False):
     """Run n_steps decode steps on the GPU from setup.state0; the oracle follows the
-    (b, h) pairs in ``sample`` (all pairs if None).  Returns max relative errors."""
+    (b, h) pairs in ``sample`` (all pairs if None).  With ``fused_gates`` the GPU forms the
+    gates inside the step (gdn_decode_step_gated).  Returns max relative errors."""
     import oracle
     import gated_deltanet_sequence_delta_b200 as G
     B, HK, HV = setup.B, setup.HK, setup.HV
@@ -23,9 +24,13 @@ def _run_steps(setup, n_steps, sample=None, check_every=1):
     worst_o = worst_s = 0.0
     for s in range(n_steps):
         q, k, v, a, b = setup.step(s)
-        g, beta = G.gdn_gates(to_dev(a), to_dev(b), A_log, dt_bias)
-        o = G.gdn_decode_step(to_dev(q), to_dev(k), to_dev(v), g, beta, state, scale=setup.scale,
-                              qk_l2norm=setup.l2norm)
+        if fused_gates:
+            o = G.gdn_decode_step_gated(to_dev(q), to_dev(k), to_dev(v), to_dev(a), to_dev(b), A_log, dt_bias,
+                                        state, scale=setup.scale, qk_l2norm=setup.l2norm)
+        else:
+            g, beta = G.gdn_gates(to_dev(a), to_dev(b), A_log, dt_bias)
+            o = G.gdn_decode_step(to_dev(q), to_dev(k), to_dev(v), g, beta, state, scale=setup.scale,
+                                  qk_l2norm=setup.l2norm)
         g_ref, beta_ref = oracle.gates(a.astype(np.float64), b.astype(np.float64),
                                        setup.A_log.astype(np.float64), setup.dt_bias.astype(np.float64))
         bi = np.array([p[0] for p in pairs])
@@ -74,6 +79,37 @@ def test_decode_workload_all_steps_sampled():
     pairs = sorted({(int(rng.integers(64)), int(rng.integers(32))) for _ in range(12)} | {(0, 0), (63, 31)})
     _run_steps(setup, I.DECODE_STEPS, sample=pairs, check_every=64)
     import gated_deltanet_sequence_delta_b200 as G
+    assert G.gdn_decode_status() == 0
+
+
+@pytest.mark.parametrize("io,ab", [(I.BF16, I.BF16), (I.BF16, I.F32), (I.F32, I.F32)])
+@pytest.mark.parametrize("D", [128, 64])
+def test_decode_gated_equals_gates_then_step(io, ab, D):
+    """The fused-gate step is bit-identical to gdn_gates followed by gdn_decode_step."""
+    import torch
+    import gated_deltanet_sequence_delta_b200 as G
+    setup = I.decode(B=5, H=8, D=D, io_dtype=io, seed=17, HK=4)
+    A_log, dt_bias = to_dev(setup.A_log), to_dev(setup.dt_bias)
+    st1 = to_dev(setup.state0.copy())
+    st2 = st1.clone()
+    for s in range(4):
+        q, k, v, a, b = setup.step(s)
+        da, db = to_dev(a), to_dev(b)
+        if ab == I.BF16:
+            da, db = da.to(torch.bfloat16), db.to(torch.bfloat16)
+        g, beta = G.gdn_gates(da, db, A_log, dt_bias)
+        o1 = G.gdn_decode_step(to_dev(q), to_dev(k), to_dev(v), g, beta, st1, scale=setup.scale)
+        o2 = G.gdn_decode_step_gated(to_dev(q), to_dev(k), to_dev(v), da, db, A_log, dt_bias, st2,
+                                     scale=setup.scale)
+        assert torch.equal(o1, o2), f"step {s}: o differs"
+        assert torch.equal(st1, st2), f"step {s}: state differs"
+
+
+def test_decode_gated_workload_vs_oracle():
+    """B=64, H=32, d=128, bf16, gates fused: 16 steps on every (sequence, head)."""
+    import gated_deltanet_sequence_delta_b200 as G
+    setup = I.decode()
+    _run_steps(setup, 16, fused_gates=True)
     assert G.gdn_decode_status() == 0
 
 
