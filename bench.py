@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "GDN prefill tokens/s @32K,H32,d128; decode-step HBM GB/s vs peak"
 PREFILL = dict(B=1, T=32768, HK=16, HV=32, D=128, BT=64)
 DECODE = dict(B=64, H=32, D=128, steps=1024)
+E2E_PIECE = 4096   # tokens per piece of the host-buffer pipeline (8 pieces at T = 32768)
 WORKLOAD = "long prefill: B=1 T=32768 HK=16 HV=32 Dk=Dv=128 bf16 BT=64, fp32 state, zero initial state"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -320,22 +321,22 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     kernel_ms = max_over_ranks(kernel_ms_local)
 
     # ---------------- e2e through host buffers ----------------
+    # gdn_chunk_prefill_host: host q, k, v, a, b (and the two per-head gate parameters) in,
+    # host o and final state out; the library streams the sequence through the GPU in
+    # pieces so that the copies in both directions overlap the kernels.
     hq, hk_, hv = pinned(inp.q), pinned(inp.k), pinned(inp.v)
-    ha, hb = pinned(inp.a), pinned(inp.b)
+    ha, hb = pinned(inp.a).view(1, T, HV), pinned(inp.b).view(1, T, HV)
+    hAl, hdtb = pinned(inp.A_log), pinned(inp.dt_bias)
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hh = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk_, hv, ha, hb))
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk_, hv, ha, hb, hAl, hdtb))
     d2h = ho.numel() * ho.element_size() + hh.numel() * hh.element_size()
+    hws = torch.empty(G.prefill_host_workspace_bytes(1, T, HK, HV, D, D, BT, 1, 0, E2E_PIECE),
+                      dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk_, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        a.copy_(ha, non_blocking=True)
-        b.copy_(hb, non_blocking=True)
-        prefill_step()
-        ho.copy_(o, non_blocking=True)
-        hh.copy_(hT, non_blocking=True)
+        G.gdn_chunk_prefill_host(hq, hk_, hv, ha, hb, hAl, hdtb, BT=BT, piece_tokens=E2E_PIECE, o=ho,
+                                 final_state=hh, workspace=hws)
 
     for _ in range(2):
         e2e_step()
@@ -349,7 +350,7 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     e1.record()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
-    del hq, hk_, hv, ha, hb, ho, hh
+    del hq, hk_, hv, ha, hb, hAl, hdtb, ho, hh, hws
     flops = prefill_flops_per_token(HK, HV, D, BT) * T
     pbytes = prefill_bytes_per_token(HK, HV, D) * T + HV * D * D * 4
     tflops = flops / (kernel_ms * 1e-3) / 1e12
@@ -368,7 +369,8 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
                                   "frac": pbytes / (kernel_ms * 1e-3) / 1e9 / P["hbm_gbs"],
                                   "bytes_per_launch": pbytes}},
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "path": f"gdn_chunk_prefill_host, pinned host buffers, {E2E_PIECE}-token pieces"},
         "gpu_launches": launches,
     }
 

@@ -49,6 +49,11 @@ _SIGS = {
     "gdn_decode_step": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                          _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_chunk_prefill_host_workspace_bytes": ([_i32, _i64, _i32, _i32, _i32, _i32, _i32, ctypes.c_int,
+                                                ctypes.c_int, _i64], _sz),
+    "gdn_chunk_prefill_host": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i64,
+                                _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i64, _vp, _vp, _vp, _sz, _vp],
+                               ctypes.c_int),
     "gdn_decode_step_gated": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32,
                                _i32, _i32, _i32, _f32, _i32, _vp, _vp], ctypes.c_int),
 }
@@ -114,6 +119,15 @@ def _ptr(t: torch.Tensor | None):
         raise ValueError("tensors must be CUDA tensors")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _hptr(t: torch.Tensor | None):
+    """Address of a contiguous host (CPU) tensor, None for None."""
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("host tensors must be contiguous CPU tensors")
     return t.data_ptr()
 
 
@@ -229,6 +243,46 @@ def gdn_decode_step_gated(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1
                                      int(bool(qk_l2norm)), _ptr(o), _stream())
     _check(st, "gdn_decode_step_gated")
     return o
+
+
+def prefill_host_workspace_bytes(B, T, HK, HV, Dk, Dv, BT, io_dtype, ab_dtype, piece_tokens) -> int:
+    return int(lib().gdn_chunk_prefill_host_workspace_bytes(B, T, HK, HV, Dk, Dv, BT, io_dtype, ab_dtype,
+                                                            piece_tokens))
+
+
+def gdn_chunk_prefill_host(q, k, v, a, b, A_log, dt_bias, initial_state=None, BT: int = 64, scale: float = 1.0,
+                           qk_l2norm: bool = True, piece_tokens: int = 4096, o=None, final_state=None,
+                           workspace=None):
+    """Gates + chunked prefill for host (CPU) tensors, pipelined through the GPU in pieces
+    of ``piece_tokens`` tokens: q, k [B, T, HK, Dk]; v [B, T, HV, Dv]; a, b [B, T, HV];
+    A_log, dt_bias [HV]; initial_state [B, HV, Dk, Dv] or None.  Returns host tensors
+    (o, final_state).  Pinned host memory lets the copies overlap; the call synchronises
+    nothing but the current stream waits for all of it."""
+    B, T, HK, Dk = q.shape
+    HV, Dv = v.shape[-2:]
+    for t in (q, k, v, a, b, A_log, dt_bias):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host inputs must be contiguous CPU tensors")
+    if k.shape != q.shape or v.shape[:2] != (B, T) or a.shape != (B, T, HV) or b.shape != (B, T, HV):
+        raise ValueError("inconsistent prefill shapes")
+    if A_log.dtype != torch.float32 or dt_bias.dtype != torch.float32 or a.dtype != b.dtype:
+        raise ValueError("A_log, dt_bias must be fp32; a, b must share a dtype")
+    io, ab = _dtype_code(q), _dtype_code(a)
+    if o is None:
+        o = torch.empty((B, T, HV, Dv), dtype=q.dtype).pin_memory()
+    if final_state is None:
+        final_state = torch.empty((B, HV, Dk, Dv), dtype=torch.float32).pin_memory()
+    need = prefill_host_workspace_bytes(B, T, HK, HV, Dk, Dv, BT, io, ab, piece_tokens)
+    if need == 0:
+        raise GDNError(4, "gdn_chunk_prefill_host: unsupported sizes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    st = lib().gdn_chunk_prefill_host(_hptr(q), _hptr(k), _hptr(v), io, _hptr(a), _hptr(b), ab, _hptr(A_log),
+                                      _hptr(dt_bias), _hptr(initial_state), B, T, HK, HV, Dk, Dv, BT, float(scale),
+                                      int(bool(qk_l2norm)), int(piece_tokens), _hptr(o), _hptr(final_state),
+                                      _ptr(workspace), workspace.numel(), _stream())
+    _check(st, "gdn_chunk_prefill_host")
+    return o, final_state
 
 
 def gdn_decode_status() -> int:

@@ -192,6 +192,42 @@ GDN_API gdn_status gdn_chunk_prefill_static_ws(const void* q, const void* k, con
                              void* o, float* final_state, void* stream);
 
 /*
+ * gdn_chunk_prefill_host -- gdn_gates followed by gdn_chunk_prefill for inputs and outputs
+ * that live in HOST memory.  The sequences are streamed through the GPU in pieces of
+ * `piece_tokens` tokens (a multiple of BT): the host -> device copies of one piece, the
+ * kernels of the previous piece and the device -> host copies of the one before overlap
+ * on three library-owned streams with two buffer slots each way, and the state is carried
+ * between pieces in place on the device.  The pages have no counterpart of this call; it
+ * is the runtime around the chunked form of the "QWEN3.5" Q&A page, question 1 (chunks in
+ * order, the state carried serially), for callers whose data arrives from the host.
+ *   q, k   [B, T, HK, Dk] io_dtype;  v [B, T, HV, Dv] io_dtype      (host, read)
+ *   a, b   [B, T, HV] ab_dtype;  A_log, dt_bias [HV] fp32            (host, read)
+ *   initial_state [B, HV, Dk, Dv] fp32 or NULL (zeros)              (host, read)
+ *   o      [B, T, HV, Dv] io_dtype                                  (host, written)
+ *   final_state [B, HV, Dk, Dv] fp32 or NULL                        (host, written)
+ *   workspace   device, 256-byte aligned, gdn_chunk_prefill_host_workspace_bytes() bytes
+ * Dense sequences only (no cu_seqlens).  Results equal gdn_chunk_prefill's up to the
+ * rounding of the fp16 intermediates, whose power-of-two scale is chosen per piece.
+ * Asynchronous: returns once the work is enqueued; `stream` waits for all of it, so the
+ * host buffers must stay valid until `stream` reaches that point, and page-locked host
+ * memory is needed for the copies to overlap.  The internal streams and events are
+ * created on the first call on a device and kept for the life of the process; calls on
+ * one device are serialised.  Not for use inside a CUDA graph capture.
+ * Errors: NULL, SHAPE (piece_tokens <= 0 or not a multiple of BT), UNSUPPORTED, ALIGN
+ * (workspace), WORKSPACE, CUDA, or any error of the two calls it makes.
+ */
+GDN_API size_t gdn_chunk_prefill_host_workspace_bytes(int32_t B, int64_t T, int32_t HK, int32_t HV,
+                             int32_t Dk, int32_t Dv, int32_t BT, gdn_dtype io_dtype, gdn_dtype ab_dtype,
+                             int64_t piece_tokens);
+GDN_API gdn_status gdn_chunk_prefill_host(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                             const void* a, const void* b, gdn_dtype ab_dtype,
+                             const float* A_log, const float* dt_bias, const float* initial_state,
+                             int32_t B, int64_t T, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                             int32_t BT, float scale, int32_t qk_l2norm, int64_t piece_tokens,
+                             void* o, float* final_state, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/*
  * gdn_decode_step -- one token per sequence, state updated in place (the
  * incremental update of the "QWEN3.5" Q&A page, question 2a: decay the whole
  * state by alpha, then clear and write along the current key with strength beta).

@@ -126,6 +126,33 @@ def test_decode_gated_validation(L):
     assert call(a10=0) == 0                     # B = 0: nothing to do
 
 
+def test_prefill_host_validation(L):
+    f = L.gdn_chunk_prefill_host
+    ws_need = L.gdn_chunk_prefill_host_workspace_bytes(1, 1000, 2, 4, 128, 128, 64, 1, 0, 256)
+    assert ws_need > 0
+    assert L.gdn_chunk_prefill_host_workspace_bytes(1, 1000, 2, 4, 128, 128, 64, 1, 0, 100) == 0   # piece % BT
+    assert L.gdn_chunk_prefill_host_workspace_bytes(1, 1000, 2, 4, 32, 128, 64, 1, 0, 256) == 0    # head dim
+    # q, k, v, io, a, b, ab, A_log, dt_bias, h0, B, T, HK, HV, Dk, Dv, BT, scale, l2, piece, o, hT, ws, bytes, stream
+    base = [A, A + MB, A + 2 * MB, 1, A + 3 * MB, A + 4 * MB, 0, A + 5 * MB, A + 6 * MB, None,
+            1, 1000, 2, 4, 128, 128, 64, 1.0, 1, 256, A + 8 * MB, A + 9 * MB, A + 16 * MB, ws_need, None]
+    def call(**kw):
+        a = list(base)
+        for i, val in kw.items():
+            a[int(i[1:])] = val
+        return f(*a)
+    assert call(a19=100) == 2                   # piece not a multiple of BT
+    assert call(a19=0) == 2
+    assert call(a13=3) == 2                     # HV % HK
+    assert call(a14=32) == 4                    # head dim
+    assert call(a6=9) == 4                      # ab dtype
+    assert call(a0=None) == 1
+    assert call(a8=None) == 1
+    assert call(a22=None) == 6                  # no workspace
+    assert call(a23=ws_need - 1) == 6           # workspace too small
+    assert call(a22=A + 16 * MB + 16) == 3      # workspace not 256-byte aligned
+    assert call(a10=0) == 0                     # B = 0: nothing to do
+
+
 def test_decode_status_null(L):
     assert L.gdn_decode_status(None) == 1
 
