@@ -38,6 +38,47 @@ WORKLOAD = "long prefill: B=1 T=32768 HK=16 HV=32 Dk=Dv=128 bf16 BT=64, fp32 sta
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+class RankOps:
+    """The cross-rank steps of a run: a barrier and the max over ranks of a time.  With
+    ``dist`` None (one process) both are local.  With a process group they are
+    collectives (NCCL between GPUs; gloo in the CPU tests), and every rank takes them in
+    the same order.  No data of the path itself crosses ranks: each rank runs an
+    independent replica of the workload (seed ``replica_seed``)."""
+
+    def __init__(self, dist=None, device=None):
+        self.dist = dist
+        self.device = device
+
+    def _sync(self):
+        if self.device is not None and getattr(self.device, "type", "cpu") == "cuda":
+            import torch
+            torch.cuda.synchronize()
+
+    def barrier(self):
+        self._sync()
+        if self.dist is not None:
+            self.dist.barrier()
+        self._sync()
+
+    def max(self, x: float) -> float:
+        if self.dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Seed of rank ``rank``'s replica of a workload whose single-GPU seed is ``base``."""
+    return base + 1000 * rank
+
+
+def whole_job_rate(world: int, units_per_rank: int, ms_max: float) -> float:
+    """Units per second over all ranks, timed by the slowest rank."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -229,18 +270,8 @@ def run_gdn(args, rank, world, dist):
             return torch.from_numpy(t.data).pin_memory()
         return torch.from_numpy(np.ascontiguousarray(t)).pin_memory()
 
-    def barrier():
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ops = RankOps(dist, dev)
+    barrier, max_over_ranks = ops.barrier, ops.max
 
     T, HK, HV, D, BT = PREFILL["T"], PREFILL["HK"], PREFILL["HV"], PREFILL["D"], PREFILL["BT"]
     do_prefill = args.only in ("all", "prefill")
@@ -281,7 +312,7 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     import gated_deltanet_sequence_delta_b200 as G
     from gated_deltanet_sequence_delta_b200 import inputs as I
     T, HK, HV, D, BT = PREFILL["T"], PREFILL["HK"], PREFILL["HV"], PREFILL["D"], PREFILL["BT"]
-    inp = I.make_prefill(1, T, HK, HV, D, D, io_dtype=I.BF16, seed=2 + 1000 * rank, BT=BT, name="long")
+    inp = I.make_prefill(1, T, HK, HV, D, D, io_dtype=I.BF16, seed=replica_seed(2, rank), BT=BT, name="long")
     q, k, v = dev_t(inp.q), dev_t(inp.k), dev_t(inp.v)
     a, b = dev_t(inp.a), dev_t(inp.b)
     A_log, dt_bias = dev_t(inp.A_log), dev_t(inp.dt_bias)
@@ -356,7 +387,7 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     tflops = flops / (kernel_ms * 1e-3) / 1e12
     peak_tf = P["bf16_tflops"]
     return {
-        "value": world * T / (ms * 1e-3), "ms_per_step": ms,
+        "value": whole_job_rate(world, T, ms), "ms_per_step": ms,
         "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": T,
                    "l2": "no flush: each step reads/writes ~0.8 GB, over 6x the 126 MB L2",
                    "parallelism": f"replicas x{world} (independent problems, no collective)"},
@@ -368,7 +399,7 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
                                   "peak_gbs": P["hbm_gbs"],
                                   "frac": pbytes / (kernel_ms * 1e-3) / 1e9 / P["hbm_gbs"],
                                   "bytes_per_launch": pbytes}},
-        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(world, T, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "path": f"gdn_chunk_prefill_host, pinned host buffers, {E2E_PIECE}-token pieces"},
         "gpu_launches": launches,
@@ -379,7 +410,7 @@ def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, 
     import torch
     import gated_deltanet_sequence_delta_b200 as G
     from gated_deltanet_sequence_delta_b200 import inputs as I
-    ds = I.decode(B=DECODE["B"], H=DECODE["H"], D=DECODE["D"], seed=1 + 1000 * rank)
+    ds = I.decode(B=DECODE["B"], H=DECODE["H"], D=DECODE["D"], seed=replica_seed(1, rank))
     ring = []
     for s in range(8):
         dq, dk, dv, da, db = ds.step(s)
