@@ -769,7 +769,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 const int st = c % NSTAGE, r = c / NSTAGE;
                 const CarryStage& B = S.st[st];
                 bool ok = tc::mbar_wait(&S.full[st], r & 1);
-                ok = ok && tc::mbar_wait(&S.h0_ready, c & 1);
+                ok = ok && tc::mbar_wait_spin(&S.h0_ready, c & 1);
                 if (!ok || S.abort) {
                     if (!ok) record_timeout(status);
                     S.abort = 1;
@@ -785,7 +785,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                     tc::mma_bf16(tA + par, da + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
                                  dh + (uint64_t)((kk * 2 * kOpLBO) >> 4), idA, kk > 0);
                 tc::mma_commit(&S.bar_a);
-                if (!tc::mbar_wait(&S.d_ready, c & 1) || S.abort) {
+                if (!tc::mbar_wait_spin(&S.d_ready, c & 1) || S.abort) {
                     record_timeout(status);
                     S.abort = 1;
                     break;

@@ -44,6 +44,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
         : "memory");
     return done != 0;
 }
+__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// The same wait for a hand-off on a serial chain: polls with the non-suspending test
+// first (no wake-up delay), then falls back to mbar_wait's bounded wait.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = 2000000000ull);
+
 // Wait for the phase with the given parity to complete; give up after `timeout_ns`
 // of wall time (returns false).  Never spins forever.  The first ~20 us poll without
 // sleeping (a sleep can oversleep a short wait by far more than the wait itself).
@@ -61,6 +76,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
         if (dt > timeout_ns) return false;
         if (dt > 20000) __nanosleep(256);
     }
+}
+
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+    const uint32_t addr = smem_u32(bar);
+    for (int i = 0; i < 4096; ++i)
+        if (mbar_test_wait(addr, parity)) return true;
+    return mbar_wait(bar, parity, timeout_ns);
 }
 
 // ---- proxies and TMEM ordering fences ------------------------------------------------
