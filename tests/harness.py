@@ -108,28 +108,31 @@ def oracle_prefill(inp, heads=None):
     """Oracle o [B, T, len(heads), Dv] and hT [N, len(heads), Dk, Dv] for the given
     value heads (all heads by default)."""
     import oracle
-    heads = list(range(inp.HV)) if heads is None else list(heads)
-    G_ = inp.HV // inp.HK
     g, beta = oracle_gates(inp)
     cu = None if inp.cu_seqlens is None else inp.cu_seqlens.astype(np.int64)
-    os_, hs = [], []
-    for h in heads:
-        hk = h // G_
-        q = inp.q.f64((slice(None), slice(None), slice(hk, hk + 1)))
-        k = inp.k.f64((slice(None), slice(None), slice(hk, hk + 1)))
-        v = inp.v.f64((slice(None), slice(None), slice(h, h + 1)))
-        h0 = None if inp.h0 is None else inp.h0[:, h:h + 1].astype(np.float64)
-        gh = g[:, :, h:h + 1]
-        bh = beta[:, :, h:h + 1]
+    if heads is None or list(heads) == list(range(inp.HV)):
+        # every head in one call: the oracle spreads (sequence, head) pairs over the host cores
+        q, k, v = inp.q.f64(), inp.k.f64(), inp.v.f64()
+        h0 = None if inp.h0 is None else inp.h0.astype(np.float64)
         if cu is None:
-            o, hT = oracle.recurrence(q, k, v, gh, bh, h0=h0, scale=inp.scale, l2norm=inp.l2norm)
-        else:
-            o, hT = oracle.recurrence(q[0], k[0], v[0], gh[0], bh[0], h0=h0, cu_seqlens=cu,
-                                      scale=inp.scale, l2norm=inp.l2norm)
-            o = o[None]
-        os_.append(o)
-        hs.append(hT)
-    return np.concatenate(os_, axis=2), np.concatenate(hs, axis=1)
+            return oracle.recurrence(q, k, v, g, beta, h0=h0, scale=inp.scale, l2norm=inp.l2norm)
+        o, hT = oracle.recurrence(q[0], k[0], v[0], g[0], beta[0], h0=h0, cu_seqlens=cu, scale=inp.scale,
+                                  l2norm=inp.l2norm)
+        return o[None], hT
+    # selected heads: each value head with its own copy of its q/k head, all in one call
+    heads = list(heads)
+    G_ = inp.HV // inp.HK
+    kh = [h // G_ for h in heads]
+    q = inp.q.f64((slice(None), slice(None), kh))
+    k = inp.k.f64((slice(None), slice(None), kh))
+    v = inp.v.f64((slice(None), slice(None), heads))
+    h0 = None if inp.h0 is None else inp.h0[:, heads].astype(np.float64)
+    gs, bs = g[:, :, heads], beta[:, :, heads]
+    if cu is None:
+        return oracle.recurrence(q, k, v, gs, bs, h0=h0, scale=inp.scale, l2norm=inp.l2norm)
+    o, hT = oracle.recurrence(q[0], k[0], v[0], gs[0], bs[0], h0=h0, cu_seqlens=cu, scale=inp.scale,
+                              l2norm=inp.l2norm)
+    return o[None], hT
 
 
 def check_prefill(inp, heads=None, BT=None, tol=None):

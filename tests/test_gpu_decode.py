@@ -71,6 +71,15 @@ def test_decode_workload_first_steps_all_heads():
     assert G.gdn_decode_status() == 0   # no bounded wait expired
 
 
+def test_decode_workload_all_steps_all_heads():
+    """All 1024 steps of the B=64, H=32, d=128 workload on every (sequence, head), checked
+    every 64 steps and at the end."""
+    import gated_deltanet_sequence_delta_b200 as G
+    setup = I.decode()
+    _run_steps(setup, I.DECODE_STEPS, check_every=64)
+    assert G.gdn_decode_status() == 0
+
+
 def test_decode_workload_all_steps_sampled():
     """All 1024 steps of the B=64, H=32, d=128 workload; the oracle follows 12
     sampled (sequence, head) pairs, checked every 64 steps and at the end."""
