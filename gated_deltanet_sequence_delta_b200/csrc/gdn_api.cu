@@ -89,7 +89,7 @@ gdn_status gdn_gates(const void* a, const void* b, gdn_dtype ab_dtype, const flo
 
 size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seqs, int32_t HK, int32_t HV,
                                          int32_t Dk, int32_t Dv, int32_t BT, gdn_dtype io_dtype) {
-    if (n_tokens < 0 || n_seqs < 0 || HK <= 0 || HV <= 0 || HV % HK != 0) return 0;
+    if (n_tokens < 0 || n_tokens > INT32_MAX || n_seqs < 0 || HK <= 0 || HV <= 0 || HV % HK != 0) return 0;
     if (!head_dim_ok(Dk) || !head_dim_ok(Dv) || !dtype_ok(io_dtype)) return 0;
     if (!(BT == 16 || BT == 32 || BT == 64)) return 0;
     if (io_dtype == GDN_BF16 && BT != 64) return 0;

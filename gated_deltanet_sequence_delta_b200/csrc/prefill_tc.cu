@@ -1001,6 +1001,9 @@ bool prefill_tc_supported(int Dk, int Dv, int HK, int HV, int BT) {
 }
 
 size_t prefill_tc_workspace_bytes(int64_t n_tokens, int n_seqs, int HK, int HV) {
+    // TMA coordinates are 32-bit: token index, tile rows (chunk, head) * 64 and * 128
+    const int64_t max_chunks = (n_tokens + C - 1) / C + n_seqs;
+    if (n_tokens > INT32_MAX || max_chunks * HV * 64 > INT32_MAX || max_chunks * HK * 128 > INT32_MAX) return 0;
     return tc_layout(n_tokens, n_seqs, HK, HV).total;
 }
 

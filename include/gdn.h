@@ -97,7 +97,8 @@ GDN_API gdn_status gdn_gates(const void* a, const void* b, gdn_dtype ab_dtype,
 /*
  * Workspace size in bytes that gdn_chunk_prefill needs for these sizes (always
  * >= 256: the first 256 bytes hold the device status word).  Returns 0 for
- * sizes that gdn_chunk_prefill would reject.
+ * sizes that gdn_chunk_prefill would reject, including totals past the 32-bit
+ * coordinates of the tile copies (over 2^31 - 1 tokens, or chunks x heads x 64 rows).
  */
 GDN_API size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seqs,
                                          int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,

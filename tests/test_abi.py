@@ -73,6 +73,10 @@ def test_prefill_workspace_query(L):
     assert L.gdn_chunk_prefill_workspace_bytes(256, 1, 2, 2, 64, 64, 64, 0) >= 256
     assert L.gdn_chunk_prefill_workspace_bytes(256, 1, 2, 3, 64, 64, 64, 0) == 0
     assert L.gdn_chunk_prefill_workspace_bytes(256, 1, 2, 2, 80, 64, 64, 0) == 0
+    # beyond the 32-bit coordinates of the tile copies
+    assert L.gdn_chunk_prefill_workspace_bytes(2 ** 31, 1, 16, 32, 128, 128, 64, 1) == 0
+    assert L.gdn_chunk_prefill_workspace_bytes(2 ** 26, 1, 32, 32, 128, 128, 64, 1) == 0
+    assert L.gdn_chunk_prefill_workspace_bytes(2 ** 20, 1, 32, 32, 128, 128, 64, 1) > 0
 
 
 def test_gates_validation(L):
