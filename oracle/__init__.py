@@ -20,6 +20,9 @@ Public functions (all fp64 numpy in, fp64 numpy out):
 * ``decode_step(q, k, v, g, beta, state, ...) -> (o, new_state)`` -- the same
   recurrence for one token per sequence, the incremental update of the
   "QWEN3.5" Q&A page (question 2a).
+* ``conv(x, w, state=None, act=0) -> (y, new_state)`` -- the causal depthwise
+  convolution of kernel 4 that the Qwen3-next page (section 3.1) puts before the
+  gated update, with its rolling state of the three previous inputs.
 """
 from __future__ import annotations
 
@@ -77,6 +80,9 @@ class OracleLib:
             ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
             ctypes.c_int, _dp, _dp, ctypes.c_int]
         lib.gdn_oracle_recurrence.restype = ctypes.c_int
+        lib.gdn_oracle_conv.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_int, _dp, _dp]
+        lib.gdn_oracle_conv.restype = None
         lib.gdn_oracle_max_threads.argtypes = []
         lib.gdn_oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
@@ -146,6 +152,24 @@ class OracleLib:
             raise ValueError(f"gdn_oracle_recurrence failed with code {rc}")
         return o.reshape(out_shape), hT
 
+    # -- convolution prologue --------------------------------------------
+    def conv(self, x, w, state=None, act: int = 0):
+        """x [B, T, C]; w [C, 4] (taps oldest first); state [B, C, 3] or None.
+        Returns (y [B, T, C], new state [B, C, 3])."""
+        x = _f64(x)
+        w = _f64(w)
+        if x.ndim != 3 or w.shape != (x.shape[2], 4):
+            raise ValueError("conv: x must be [B, T, C] and w [C, 4]")
+        B, T, C = x.shape
+        if state is not None:
+            state = _f64(state)
+            if state.shape != (B, C, 3):
+                raise ValueError("conv: state must be [B, C, 3]")
+        y = np.empty_like(x)
+        new_state = np.empty((B, C, 3))
+        self.lib.gdn_oracle_conv(_ptr(x), _ptr(w), _ptr(state), B, T, C, int(act), _ptr(y), _ptr(new_state))
+        return y, new_state
+
     def decode_step(self, q, k, v, g, beta, state, scale: float = 1.0,
                     l2norm: bool = True, threads: int = 0):
         """One token per sequence: q, k [B, HK, Dk]; v [B, HV, Dv];
@@ -176,6 +200,10 @@ def recurrence(q, k, v, g, beta, h0=None, cu_seqlens=None, scale=1.0,
                l2norm=True, threads=0):
     return default().recurrence(q, k, v, g, beta, h0=h0, cu_seqlens=cu_seqlens,
                                 scale=scale, l2norm=l2norm, threads=threads)
+
+
+def conv(x, w, state=None, act=0):
+    return default().conv(x, w, state=state, act=act)
 
 
 def decode_step(q, k, v, g, beta, state, scale=1.0, l2norm=True, threads=0):

@@ -32,6 +32,16 @@
  *   - packed sequences: tokens cu_seqlens[n] .. cu_seqlens[n+1]-1 form
  *     sequence n, each with its own initial state.
  *
+ *   Convolution prologue (the Qwen3-next page, section 3.1, names a depthwise
+ *   separable convolution before the gated update; the tutorial page, section 6,
+ *   gives its kernel size field linear_conv_kernel_dim = 4):
+ *       y_t[c] = act( sum_{i=0..3} w[c][i] * x_{t-3+i}[c] )
+ *   per channel c, causal, with x_{-3..-1} taken from a per-sequence state of
+ *   the three previous inputs (zeros if none) and the state after the last token
+ *   the three last inputs.  Readings: the taps run oldest to newest; the pages
+ *   name no activation, so act is the identity or, on request, SiLU
+ *   (x * sigmoid(x)).
+ *
  * Everything is fp64.  No blocking, chunking or reordering: one token at a
  * time, exactly the formula above.  OpenMP only splits independent
  * (sequence, value head) pairs across threads.
@@ -168,6 +178,32 @@ int gdn_oracle_recurrence(const double* q, const double* k, const double* v,
 }
 
 /* Number of threads OpenMP would use (1 without OpenMP). */
+/* Causal depthwise convolution of kernel 4 over B sequences of T tokens and C
+ * channels.  x: [B, T, C]; w: [C, 4]; state_in: [B, C, 3] (oldest first) or NULL
+ * for zeros; act 0 identity, 1 SiLU.  Outputs y: [B, T, C], state_out: [B, C, 3]. */
+void gdn_oracle_conv(const double* x, const double* w, const double* state_in,
+                     int64_t B, int64_t T, int64_t C, int act,
+                     double* y, double* state_out) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t c = 0; c < C; ++c) {
+            double win[4];   /* x_{t-3}, x_{t-2}, x_{t-1}, x_t */
+            for (int i = 0; i < 3; ++i)
+                win[i] = state_in ? state_in[(b * C + c) * 3 + i] : 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                win[3] = x[(b * T + t) * C + c];
+                double acc = 0.0;
+                for (int i = 0; i < 4; ++i) acc += w[c * 4 + i] * win[i];
+                y[(b * T + t) * C + c] = act == 1 ? acc * oracle_sigmoid(acc) : acc;
+                win[0] = win[1];
+                win[1] = win[2];
+                win[2] = win[3];
+            }
+            for (int i = 0; i < 3; ++i) state_out[(b * C + c) * 3 + i] = win[i];
+        }
+    }
+}
+
 int gdn_oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

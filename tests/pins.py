@@ -14,7 +14,10 @@ rests on; none re-types the oracle's loop:
   1/2 ||S k - v||^2 after weight decay, with the gradient taken numerically;
 * a brute-force expanded product of the per-token transition matrices;
 * structural facts: linearity in (v, S0), contraction bound, independence of
-  packed sequences, grouped-head mapping, state carry, the chunked algebra.
+  packed sequences, grouped-head mapping, state carry, the chunked algebra;
+* the convolution prologue: a hand-worked example (``golden/conv_hand.json``),
+  the impulse response, the state as the three past inputs, state carry,
+  linearity, and SiLU against scipy's logistic function.
 """
 from __future__ import annotations
 
@@ -368,10 +371,87 @@ def pin_chunked_algebra(orc):
         np.testing.assert_allclose(hc, hT, rtol=1e-10, atol=1e-11)
 
 
+# ---------------------------------------------------------------------------
+# the convolution prologue (Qwen3-next page, section 3.1; kernel size 4 from the
+# tutorial page, section 6)
+# ---------------------------------------------------------------------------
+def pin_conv_hand(orc):
+    """A two-channel, three-token example with a non-zero state, worked by hand."""
+    d = json.load(open(os.path.join(GOLDEN, "conv_hand.json")))
+    y, st = orc.conv(np.array(d["x"])[None], np.array(d["w"]), np.array(d["state"])[None])
+    np.testing.assert_array_equal(y[0], np.array(d["y"]))
+    np.testing.assert_array_equal(st[0], np.array(d["state_out"]))
+
+
+def pin_conv_impulse_response(orc):
+    """A unit impulse at t = 0 from a zero state returns the taps newest first:
+    y_t = w[3 - t] for t < 4, then 0 (causality and tap order)."""
+    rng = _rng(61)
+    C = 3
+    w = rng.standard_normal((C, 4))
+    x = np.zeros((1, 7, C))
+    x[0, 0, :] = 1.0
+    y, st = orc.conv(x, w)
+    for t in range(7):
+        want = w[:, 3 - t] if t < 4 else np.zeros(C)
+        np.testing.assert_array_equal(y[0, t], want)
+    np.testing.assert_array_equal(st[0], np.zeros((C, 3)))
+
+
+def pin_conv_state_is_past_input(orc):
+    """The state stands for the three inputs before the first token: a call with
+    state s equals a zero-state call on [s; x] without its first three outputs, and
+    its returned state is the last three inputs."""
+    rng = _rng(62)
+    B, T, C = 2, 9, 4
+    w = rng.standard_normal((C, 4))
+    s = rng.standard_normal((B, C, 3))
+    x = rng.standard_normal((B, T, C))
+    y, st = orc.conv(x, w, s)
+    xx = np.concatenate([np.transpose(s, (0, 2, 1)), x], axis=1)
+    yy, _ = orc.conv(xx, w)
+    np.testing.assert_allclose(y, yy[:, 3:], rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(st, np.transpose(x[:, -3:], (0, 2, 1)))
+
+
+def pin_conv_state_carry(orc):
+    """One call over T tokens equals two calls over the two halves with the state carried."""
+    rng = _rng(63)
+    B, T, C = 2, 11, 5
+    w = rng.standard_normal((C, 4))
+    x = rng.standard_normal((B, T, C))
+    s0 = rng.standard_normal((B, C, 3))
+    for act in (0, 1):
+        y, st = orc.conv(x, w, s0, act)
+        y1, s1 = orc.conv(x[:, :4], w, s0, act)
+        y2, s2 = orc.conv(x[:, 4:], w, s1, act)
+        np.testing.assert_array_equal(y, np.concatenate([y1, y2], axis=1))
+        np.testing.assert_array_equal(st, s2)
+
+
+def pin_conv_linear_and_silu(orc):
+    """Without an activation the convolution is linear in (x, state); SiLU is the
+    identity output times scipy's logistic sigmoid of it."""
+    from scipy.special import expit
+    rng = _rng(64)
+    B, T, C = 1, 8, 3
+    w = rng.standard_normal((C, 4))
+    x1, x2 = rng.standard_normal((2, B, T, C))
+    s1, s2 = rng.standard_normal((2, B, C, 3))
+    y1, _ = orc.conv(x1, w, s1)
+    y2, _ = orc.conv(x2, w, s2)
+    y12, _ = orc.conv(2.0 * x1 - 3.0 * x2, w, 2.0 * s1 - 3.0 * s2)
+    np.testing.assert_allclose(y12, 2.0 * y1 - 3.0 * y2, rtol=1e-13, atol=1e-13)
+    ys, _ = orc.conv(x1, w, s1, act=1)
+    np.testing.assert_allclose(ys, y1 * expit(y1), rtol=1e-14, atol=1e-15)
+
+
 ALL_PINS = [
     pin_gates_library, pin_gates_hand, pin_gates_dt_construction, pin_hand_worked,
     pin_no_write_keeps_state, pin_orthonormal_retrieval, pin_full_write_any_decay,
     pin_sgd_step, pin_bruteforce_product, pin_reset_clears_history, pin_linearity,
     pin_contraction_bound, pin_packed_sequences_independent, pin_grouped_heads, pin_l2norm,
     pin_state_carry, pin_chunked_algebra,
+    pin_conv_hand, pin_conv_impulse_response, pin_conv_state_is_past_input, pin_conv_state_carry,
+    pin_conv_linear_and_silu,
 ]

@@ -30,6 +30,9 @@ MUTANTS = {
     "h0_transposed": ("h0[((n * HV + h) * Dk + c) * Dv + r]", "h0[((n * HV + h) * Dv + r) * Dk + c]"),
     "l2norm_eps_outside": ("1.0 / sqrt(ss + 1e-6)", "1.0 / (sqrt(ss) + 1e-6)"),
     "scale_dropped": ("ot[r] = scale * acc;", "ot[r] = acc;"),
+    "conv_taps_reversed": ("acc += w[c * 4 + i] * win[i];", "acc += w[c * 4 + 3 - i] * win[i];"),
+    "conv_state_not_shifted": ("win[1] = win[2];", "win[1] = win[3];"),
+    "conv_silu_sign": ("acc * oracle_sigmoid(acc)", "acc * oracle_sigmoid(-acc)"),
 }
 
 _CHILD = r"""
