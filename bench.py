@@ -407,6 +407,7 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
 
 
 def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, clocks):
+    import numpy as np
     import torch
     import gated_deltanet_sequence_delta_b200 as G
     from gated_deltanet_sequence_delta_b200 import inputs as I
@@ -468,6 +469,37 @@ def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, 
     clocks.window(w0, time.time())
     gated_launches = G.kernel_launches() - nf0
     gated_ms = max_over_ranks(f0.elapsed_time(f1) / n_dec)
+    # the step from raw projections: convolution (SiLU), gates and update in one launch
+    fs = I.decode_fused(B=DECODE["B"], H=DECODE["H"], D=DECODE["D"], seed=replica_seed(1, rank))
+    fring = [(dev_t(x), dev_t(a_), dev_t(b_)) for x, a_, b_ in (fs.step(s) for s in range(8))]
+    cw = dev_t(fs.conv_w)
+    cst = [dev_t(np.ascontiguousarray(fs.conv_state0.transpose(0, 2, 1))),   # tap-major [B, 3, C]
+           torch.empty((ds.B, 3, fs.C), dtype=torch.float32, device=dev)]
+
+    def fused_step(i):
+        x, a_, b_ = fring[i % len(fring)]
+        G.gdn_decode_step_fused(x, cw, cst[i % 2], a_, b_, dA, dbias, state, HK=ds.HK, conv_act=1, o=do,
+                                conv_state_out=cst[(i + 1) % 2])
+
+    for i in range(3):
+        fused_step(i)
+    barrier()
+    nc0 = G.kernel_launches()
+    c0 = torch.cuda.Event(enable_timing=True)
+    c1 = torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    c0.record()
+    for i in range(n_dec):
+        fused_step(i)
+    c1.record()
+    barrier()
+    clocks.window(w0, time.time())
+    fused_launches = G.kernel_launches() - nc0
+    fused_ms = max_over_ranks(c0.elapsed_time(c1) / n_dec)
+    fbytes = (2 * ds.B * ds.HV * ds.Dk * ds.Dv * 4          # state in and out
+              + ds.B * fs.C * 2 + 2 * ds.B * fs.C * 3 * 4   # x (bf16), convolution state in and out
+              + fs.C * 16 + ds.B * ds.HV * (2 * 4 + ds.Dv * 2) + 2 * ds.HV * 4)   # weights, a, b, o, A_log, dt_bias
+    fgbs = fbytes / (fused_ms * 1e-3) / 1e9
     dbytes = decode_bytes_per_step(ds.B, ds.HK, ds.HV, ds.Dk, ds.Dv)
     dgbs = dbytes / (dec_kernel_ms * 1e-3) / 1e9
     ggbs = dbytes / (gated_ms * 1e-3) / 1e9
@@ -476,6 +508,10 @@ def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, 
             "ms_per_step": dec_ms, "steps_per_s": world * 1e3 / dec_ms,
             "tokens_per_s": world * ds.B * 1e3 / dec_ms,
             "gpu_launches": dec_launches,
+            "fused_step": {"what": "gdn_decode_step_fused: raw q|k|v projections, kernel-4 convolution (SiLU), "
+                                   "gates and update in one launch per step",
+                           "ms_per_step": fused_ms, "steps_per_s": world * 1e3 / fused_ms, "bytes_per_step": fbytes,
+                           "achieved_gbs": fgbs, "frac": fgbs / P["hbm_gbs"], "gpu_launches": fused_launches},
             "gated_step": {"what": "gdn_decode_step_gated: gates formed in the decode kernel, one launch per step",
                            "ms_per_step": gated_ms, "steps_per_s": world * 1e3 / gated_ms,
                            "achieved_gbs": ggbs, "frac": ggbs / P["hbm_gbs"], "gpu_launches": gated_launches},

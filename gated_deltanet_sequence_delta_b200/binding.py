@@ -49,6 +49,8 @@ _SIGS = {
     "gdn_decode_step": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                          _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_decode_step_fused": ([_vp, ctypes.c_int, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_int, _vp, _vp, _vp,
+                               _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_chunk_prefill_host_workspace_bytes": ([_i32, _i64, _i32, _i32, _i32, _i32, _i32, ctypes.c_int,
                                                 ctypes.c_int, _i64], _sz),
     "gdn_chunk_prefill_host": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i64,
@@ -283,6 +285,30 @@ def gdn_chunk_prefill_host(q, k, v, a, b, A_log, dt_bias, initial_state=None, BT
                                       _ptr(workspace), workspace.numel(), _stream())
     _check(st, "gdn_chunk_prefill_host")
     return o, final_state
+
+
+def gdn_decode_step_fused(x, conv_w, conv_state_in, a, b, A_log, dt_bias, state, HK: int, conv_act: int = 1,
+                          scale: float = 1.0, qk_l2norm: bool = True, conv_state_out=None, o=None):
+    """The decode step from raw projections: x [B, C] (C = 2 HK Dk + HV Dv, q | k | v),
+    conv_w [C, 4], conv_state_in [B, 3, C] (tap-major, oldest first); a, b [B, HV];
+    A_log, dt_bias [HV]; state [B, HV, Dk, Dv] updated in place.
+    Returns (o [B, HV, Dv], conv_state_out [B, 3, C])."""
+    B, HV, Dk, Dv = state.shape
+    C = 2 * HK * Dk + HV * Dv
+    if x.shape != (B, C) or conv_w.shape != (C, 4) or conv_state_in.shape != (B, 3, C):
+        raise ValueError("inconsistent fused decode shapes")
+    if a.shape != (B, HV) or b.shape != (B, HV) or a.dtype != b.dtype:
+        raise ValueError("a, b must be [B, HV] of one dtype")
+    if conv_state_out is None:
+        conv_state_out = torch.empty_like(conv_state_in)
+    if o is None:
+        o = torch.empty((B, HV, Dv), dtype=x.dtype, device=x.device)
+    st = lib().gdn_decode_step_fused(_ptr(x), _dtype_code(x), _ptr(conv_w), _ptr(conv_state_in),
+                                     _ptr(conv_state_out), int(conv_act), _ptr(a), _ptr(b), _dtype_code(a),
+                                     _ptr(A_log), _ptr(dt_bias), _ptr(state), B, HK, HV, Dk, Dv, float(scale),
+                                     int(bool(qk_l2norm)), _ptr(o), _stream())
+    _check(st, "gdn_decode_step_fused")
+    return o, conv_state_out
 
 
 def gdn_decode_status() -> int:

@@ -21,6 +21,7 @@
 // a bulk store.  HBM then sees a steady stream of loads and stores instead of the gaps
 // between short-lived CTAs.
 #include <mutex>
+#include <type_traits>
 
 #include "gdn_internal.cuh"
 #include "tc_ptx.cuh"
@@ -161,32 +162,45 @@ constexpr int kSWarps = 16;                // compute warps: rows 8w .. 8w+7 eac
 constexpr int kSThreads = kSWarps * 32 + 32;   // + producer warp
 struct StagedSlot {
     float H[kSD * kSD];                    // the state slice, row-major as in global memory
-    __align__(16) uint8_t q[kSD * 4], k[kSD * 4], v[kSD * 4];   // raw rows (bf16 or fp32)
+    __align__(16) uint8_t q[kSD * 4], k[kSD * 4], v[kSD * 4];   // rows (io dtype, or fp32 with CONV)
 };
+struct ConvSlot {                          // CONV: this item's convolution inputs
+    __align__(16) uint8_t x[3][kSD * 4];   // raw q, k, v channel rows (io dtype)
+    float s[3][3][kSD];                    // state taps (oldest first) x (q, k, v) x channel
+};
+template <bool CONV>
 struct StagedSmem {
     StagedSlot st[kSStages];
-    float red_u[kSWarps][kSD], red_q[kSWarps][kSD];
+    // column partial sums: their own arrays, or (CONV, for room) the slot's state tile,
+    // which is free between the reads of the old rows and the writes of the new ones
+    float red[CONV ? 1 : 2][CONV ? 1 : kSWarps][CONV ? 1 : kSD];
+    ConvSlot cv[CONV ? kSStages : 1];
     float delta[kSD];
     float dot[4];
     uint64_t full[kSStages], empty[kSStages];
 };
-constexpr size_t kStagedSmemBytes = sizeof(StagedSmem) + 128;
+template <bool CONV>
+constexpr size_t staged_smem_bytes() { return sizeof(StagedSmem<CONV>) + 128; }
 
 template <typename IO>
 __device__ __forceinline__ float ld_raw(const uint8_t* p, int i) {
     return load_elem(reinterpret_cast<const IO*>(p), i);
 }
 
-template <typename IO>
+// CONV: q, k, v are not read from memory but formed from the raw projections by the
+// convolution prologue (threads 0-383, one channel each: q, k, v rows of this item), kept
+// in the slot as fp32.
+template <typename IO, bool CONV>
 __global__ void __launch_bounds__(kSThreads, 1)
 decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
-                     const DecodeGates gates, float* __restrict__ state, int n_items, int HK, int HV,
-                     float scale, int l2norm, IO* __restrict__ o) {
+                     const DecodeConv conv, const DecodeGates gates, float* __restrict__ state, int n_items,
+                     int HK, int HV, float scale, int l2norm, IO* __restrict__ o) {
+    using QT = typename std::conditional<CONV, float, IO>::type;   // element type of the q, k, v rows
     constexpr int CPL = kSD / 32;   // 4 columns per lane
     constexpr uint32_t kRowBytes = kSD * sizeof(IO);
-    constexpr uint32_t kTx = kSD * kSD * 4 + 3 * kRowBytes;
+    constexpr uint32_t kTx = kSD * kSD * 4 + 3 * kRowBytes + (CONV ? 9 * kSD * 4 : 0);
     extern __shared__ uint8_t smem_raw[];
-    StagedSmem& S = *reinterpret_cast<StagedSmem*>(
+    StagedSmem<CONV>& S = *reinterpret_cast<StagedSmem<CONV>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
@@ -216,15 +230,40 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
                 const float* src = state + (size_t)bh * kSD * kSD;
 #pragma unroll
                 for (int p = 0; p < 4; ++p) tc::bulk_load(B.H + p * 4096, src + p * 4096, 16384, &S.full[st]);
-                tc::bulk_load(B.q, q + ((size_t)b * HK + hk) * kSD, kRowBytes, &S.full[st]);
-                tc::bulk_load(B.k, k + ((size_t)b * HK + hk) * kSD, kRowBytes, &S.full[st]);
-                tc::bulk_load(B.v, v + (size_t)bh * kSD, kRowBytes, &S.full[st]);
+                if (!CONV) {
+                    tc::bulk_load(B.q, q + ((size_t)b * HK + hk) * kSD, kRowBytes, &S.full[st]);
+                    tc::bulk_load(B.k, k + ((size_t)b * HK + hk) * kSD, kRowBytes, &S.full[st]);
+                    tc::bulk_load(B.v, v + (size_t)bh * kSD, kRowBytes, &S.full[st]);
+                } else {   // x rows and state taps of the item's q, k, v channels
+                    const int64_t C = (int64_t)2 * HK * kSD + (int64_t)HV * kSD;
+                    const int64_t c0[3] = {(int64_t)hk * kSD, (int64_t)HK * kSD + (int64_t)hk * kSD,
+                                           (int64_t)2 * HK * kSD + (int64_t)h * kSD};
+                    ConvSlot& V = S.cv[st];
+                    const IO* xb = reinterpret_cast<const IO*>(conv.x) + (int64_t)b * C;
+#pragma unroll
+                    for (int sg = 0; sg < 3; ++sg) {
+                        tc::bulk_load(V.x[sg], xb + c0[sg], kRowBytes, &S.full[st]);
+#pragma unroll
+                        for (int tp = 0; tp < 3; ++tp)
+                            tc::bulk_load(V.s[tp][sg], conv.state_in + ((int64_t)b * 3 + tp) * C + c0[sg], kSD * 4,
+                                          &S.full[st]);
+                    }
+                }
             }
         }
         return;   // the producer takes part in no later barrier
     }
 
     // ---------------- 512 compute threads (named barrier 1) ------------------------------
+    // convolution channel of this thread (CONV): seg 0 / 1 / 2 = q / k / v, d its index
+    const int cseg = tid >> 7, cd = tid & (kSD - 1);
+    const int64_t C = (int64_t)2 * HK * kSD + (int64_t)HV * kSD;
+    auto conv_channel = [&](int item) -> int64_t {
+        const int bh_ = item, b_ = bh_ / HV, h_ = bh_ - b_ * HV, hk_ = h_ / (HV / HK);
+        return cseg < 2 ? (int64_t)cseg * HK * kSD + (int64_t)hk_ * kSD + cd : (int64_t)2 * HK * kSD + (int64_t)h_ * kSD + cd;
+    };
+    float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);   // this item's taps (weights), an item ahead
+    if (CONV && tid < 3 * kSD && n_mine > 0) cw = *reinterpret_cast<const float4*>(conv.w + conv_channel(blockIdx.x) * 4);
     for (int i = 0; i < n_mine; ++i) {
         const int st = i % kSStages, r = i / kSStages;
         const int bh = blockIdx.x + i * G;
@@ -237,12 +276,34 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
             if (tid == 0) atomicExch(&g_decode_error, GDN_DEVERR_TIMEOUT);
             break;
         }
+        if (CONV) {
+            if (tid < 3 * kSD) {
+                // y = w . (x_{t-3}, x_{t-2}, x_{t-1}, x_t), then the activation; the three
+                // newest inputs go to state_out (q, k channels by the group's first value head)
+                const ConvSlot& V = S.cv[st];
+                const float s0 = V.s[0][cseg][cd], s1 = V.s[1][cseg][cd], s2 = V.s[2][cseg][cd];
+                const float xc = ld_raw<IO>(V.x[cseg], cd);
+                float y = cw.x * s0 + cw.y * s1 + cw.z * s2 + cw.w * xc;
+                if (conv.act == 1) y = y / (1.f + expf(-y));
+                float* row = reinterpret_cast<float*>(cseg == 0 ? B.q : cseg == 1 ? B.k : B.v);
+                row[cd] = y;
+                const int h = bh % HV;
+                if (cseg == 2 || h % (HV / HK) == 0) {
+                    float* so = conv.state_out + (int64_t)(bh / HV) * 3 * C + conv_channel(bh);
+                    so[0] = s1;
+                    so[C] = s2;
+                    so[2 * C] = xc;
+                }
+                if (i + 1 < n_mine) cw = *reinterpret_cast<const float4*>(conv.w + conv_channel(bh + G) * 4);
+            }
+            tc::named_bar(1, kSWarps * 32);   // q, k, v of this item are in the slot
+        }
         // norms and k.q (warps 0-2), partial column sums over this warp's 8 rows
         if (warp < 3) {
             float acc = 0.f;
             for (int e = lane; e < kSD; e += 32) {
-                const float x = warp == 1 ? ld_raw<IO>(B.k, e) : ld_raw<IO>(B.q, e);
-                const float y = warp == 0 ? ld_raw<IO>(B.q, e) : ld_raw<IO>(B.k, e);
+                const float x = warp == 1 ? ld_raw<QT>(B.k, e) : ld_raw<QT>(B.q, e);
+                const float y = warp == 0 ? ld_raw<QT>(B.q, e) : ld_raw<QT>(B.k, e);
                 acc += x * y;   // warp 0: q.q, warp 1: k.k, warp 2: q.k
             }
             acc = warp_sum(acc);
@@ -254,7 +315,7 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
         for (int rr = 0; rr < 8; ++rr) {
             const int row = warp * 8 + rr;
             hv[rr] = *reinterpret_cast<const float4*>(B.H + row * kSD + lane * CPL);
-            const float kr = ld_raw<IO>(B.k, row), qr = ld_raw<IO>(B.q, row);
+            const float kr = ld_raw<QT>(B.k, row), qr = ld_raw<QT>(B.q, row);
             const float hf[4] = {hv[rr].x, hv[rr].y, hv[rr].z, hv[rr].w};
 #pragma unroll
             for (int c = 0; c < CPL; ++c) {
@@ -262,10 +323,13 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
                 pq[c] = fmaf(qr, hf[c], pq[c]);
             }
         }
+        float* red_u = CONV ? B.H : &S.red[0][0][0];
+        float* red_q = CONV ? B.H + kSWarps * kSD : &S.red[CONV ? 0 : 1][0][0];
+        if (CONV) tc::named_bar(1, kSWarps * 32);   // every old row is in registers: the tile is scratch
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
-            S.red_u[warp][lane * CPL + c] = pu[c];
-            S.red_q[warp][lane * CPL + c] = pq[c];
+            red_u[warp * kSD + lane * CPL + c] = pu[c];
+            red_q[warp * kSD + lane * CPL + c] = pq[c];
         }
         tc::named_bar(1, kSWarps * 32);
         const float rq = l2_inv(S.dot[0], l2norm);
@@ -276,10 +340,10 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
             float su = 0.f, sq = 0.f;
 #pragma unroll
             for (int w = 0; w < kSWarps; ++w) {
-                su += S.red_u[w][j];
-                sq += S.red_q[w][j];
+                su += red_u[w * kSD + j];
+                sq += red_q[w * kSD + j];
             }
-            const float delta = bt * (ld_raw<IO>(B.v, j) - alpha * su * rk);
+            const float delta = bt * (ld_raw<QT>(B.v, j) - alpha * su * rk);
             store_elem(o, (int64_t)bh * kSD + j, scale * (alpha * (sq * rq) + delta * kq));
             S.delta[j] = delta;
         }
@@ -289,7 +353,7 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr) {
             const int row = warp * 8 + rr;
-            const float kr = ld_raw<IO>(B.k, row) * rk;
+            const float kr = ld_raw<QT>(B.k, row) * rk;
             float4 x = hv[rr];
             x.x = fmaf(alpha, x.x, kr * dl.x);
             x.y = fmaf(alpha, x.y, kr * dl.y);
@@ -325,19 +389,21 @@ int staged_grid() {
     return sms[dev];
 }
 
-template <typename IO>
-cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, const DecodeGates& gates,
-                                 float* state, int B, int HK, int HV, float scale, int l2norm, void* o,
-                                 cudaStream_t s) {
+template <typename IO, bool CONV>
+cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, const DecodeConv& conv,
+                                 const DecodeGates& gates, float* state, int B, int HK, int HV, float scale,
+                                 int l2norm, void* o, cudaStream_t s) {
     const int n_items = B * HV;
     const int sms = staged_grid();
     if (sms <= 0) return cudaErrorInvalidDevice;
-    cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kStagedSmemBytes);
+    constexpr size_t smem = staged_smem_bytes<CONV>();
+    static_assert(smem <= 227 * 1024, "staged decode: shared memory over the per-block limit");
+    cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<IO, CONV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = n_items < sms ? n_items : sms;
-    decode_staged_kernel<IO><<<grid, kSThreads, kStagedSmemBytes, s>>>(
-        (const IO*)q, (const IO*)k, (const IO*)v, gates, state, n_items, HK, HV, scale, l2norm, (IO*)o);
+    decode_staged_kernel<IO, CONV><<<grid, kSThreads, smem, s>>>(
+        (const IO*)q, (const IO*)k, (const IO*)v, conv, gates, state, n_items, HK, HV, scale, l2norm, (IO*)o);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
@@ -361,9 +427,11 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16
                           float* state, int B, int HK, int HV, int Dk, int Dv, float scale, int l2norm, void* o,
                           cudaStream_t s) {
     if (B == 0) return cudaSuccess;
+    const DecodeConv none{nullptr, nullptr, nullptr, nullptr, 0};
     if (Dk == kSD && Dv == kSD)   // the API guarantees 16-byte aligned pointers
-        return bf16 ? launch_decode_staged<__nv_bfloat16>(q, k, v, gates, state, B, HK, HV, scale, l2norm, o, s)
-                    : launch_decode_staged<float>(q, k, v, gates, state, B, HK, HV, scale, l2norm, o, s);
+        return bf16 ? launch_decode_staged<__nv_bfloat16, false>(q, k, v, none, gates, state, B, HK, HV, scale,
+                                                                 l2norm, o, s)
+                    : launch_decode_staged<float, false>(q, k, v, none, gates, state, B, HK, HV, scale, l2norm, o, s);
 #define GDN_DECODE_CASE(DK_, DV_)                                                                  \
     if (Dk == DK_ && Dv == DV_)                                                                    \
         return bf16 ? launch_decode_t<DK_, DV_, __nv_bfloat16>(q, k, v, gates, state, B, HK, HV, scale, \
@@ -374,6 +442,15 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16
     GDN_DECODE_CASE(64, 64)
 #undef GDN_DECODE_CASE
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_conv(bool bf16, const DecodeConv& conv, const DecodeGates& gates, float* state, int B,
+                               int HK, int HV, float scale, int l2norm, void* o, cudaStream_t s) {
+    if (B == 0) return cudaSuccess;
+    return bf16 ? launch_decode_staged<__nv_bfloat16, true>(nullptr, nullptr, nullptr, conv, gates, state, B, HK, HV,
+                                                            scale, l2norm, o, s)
+                : launch_decode_staged<float, true>(nullptr, nullptr, nullptr, conv, gates, state, B, HK, HV, scale,
+                                                    l2norm, o, s);
 }
 
 cudaError_t read_decode_error(int32_t* out, bool reset) {

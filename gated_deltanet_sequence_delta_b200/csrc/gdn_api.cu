@@ -229,6 +229,37 @@ gdn_status gdn_decode_step_gated(const void* q, const void* k, const void* v, gd
                                           qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
 }
 
+gdn_status gdn_decode_step_fused(const void* x, gdn_dtype io_dtype, const float* conv_w, const float* conv_state_in,
+                                 float* conv_state_out, int32_t conv_act, const void* a, const void* b,
+                                 gdn_dtype ab_dtype, const float* A_log, const float* dt_bias, float* state,
+                                 int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, float scale,
+                                 int32_t qk_l2norm, void* o, void* stream) {
+    if (B < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || HV % HK != 0) return GDN_ERR_SHAPE;
+    if (!dtype_ok(io_dtype) || !dtype_ok(ab_dtype) || Dk != 128 || Dv != 128 || (conv_act != 0 && conv_act != 1))
+        return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (!x || !conv_w || !conv_state_in || !conv_state_out || !a || !b || !A_log || !dt_bias || !state || !o)
+        return GDN_ERR_NULL;
+    const void* ptrs[] = {x, conv_w, conv_state_in, conv_state_out, a, b, A_log, dt_bias, state, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t C = (size_t)2 * HK * Dk + (size_t)HV * Dv;
+    const size_t es = esize(io_dtype), eab = esize(ab_dtype);
+    const Range rx{x, (size_t)B * C * es}, rw{conv_w, C * 16}, rci{conv_state_in, (size_t)B * C * 12};
+    const Range rco{conv_state_out, (size_t)B * C * 12};
+    const Range ra{a, (size_t)B * HV * eab}, rb{b, (size_t)B * HV * eab};
+    const Range rA{A_log, (size_t)HV * 4}, rd{dt_bias, (size_t)HV * 4};
+    const Range rs{state, (size_t)B * HV * Dk * Dv * 4}, ro{o, (size_t)B * HV * Dv * es};
+    for (Range out : {rs, ro, rco})
+        for (Range in : {rx, rw, rci, ra, rb, rA, rd})
+            if (overlap(out, in)) return GDN_ERR_ALIAS;
+    if (overlap(rs, ro) || overlap(rs, rco) || overlap(ro, rco)) return GDN_ERR_ALIAS;
+    const gdn::DecodeGates gates{nullptr, nullptr, a, b, ab_dtype == GDN_BF16, A_log, dt_bias};
+    const gdn::DecodeConv conv{x, conv_w, conv_state_in, conv_state_out, conv_act};
+    return cuda_status(gdn::launch_decode_conv(io_dtype == GDN_BF16, conv, gates, state, B, HK, HV, scale,
+                                               qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
+}
+
 gdn_status gdn_decode_status(int32_t* device_error) {
     if (!device_error) return GDN_ERR_NULL;
     cudaError_t e = cudaDeviceSynchronize();

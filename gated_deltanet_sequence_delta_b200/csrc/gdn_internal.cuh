@@ -81,6 +81,22 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16
                           float* state, int B, int HK, int HV, int Dk, int Dv, float scale, int l2norm, void* o,
                           cudaStream_t s);
 
+// The convolution prologue of a decode step: q, k, v are formed in the kernel from the raw
+// projections x = [q | k | v] per sequence (C = 2 HK Dk + HV Dv channels) by a causal
+// depthwise convolution of kernel 4, taps oldest first, over the three previous inputs
+// held in state_in and the current one; state_out receives the three newest inputs.  The
+// states are tap-major, [B, 3, C], so that a warp's channels are contiguous.
+struct DecodeConv {
+    const void* x;            // [B, C] io dtype
+    const float* w;           // [C, 4]
+    const float* state_in;    // [B, 3, C]
+    float* state_out;         // [B, 3, C]
+    int act;                  // 0 identity, 1 SiLU
+};
+// Dk = Dv = 128 only.
+cudaError_t launch_decode_conv(bool bf16, const DecodeConv& conv, const DecodeGates& gates, float* state, int B,
+                               int HK, int HV, float scale, int l2norm, void* o, cudaStream_t s);
+
 // Read (and on request clear) the device word a staged decode launch sets on a timeout.
 cudaError_t read_decode_error(int32_t* out, bool reset);
 

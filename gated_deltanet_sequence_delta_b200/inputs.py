@@ -271,3 +271,35 @@ def decode(B: int = 64, H: int = 32, D: int = 128, io_dtype: str = BF16, seed: i
 
 
 DECODE_STEPS = 1024
+
+
+@dataclass
+class FusedDecodeSetup:
+    """A decode workload fed by raw projections: per step x [B, C] with C = 2 HK Dk +
+    HV Dv (q | k | v channels), a, b [B, HV]; a kernel-4 convolution with weights
+    conv_w [C, 4] ~ N(0, 0.5^2) and an initial convolution state conv_state0 [B, C, 3]
+    ~ N(0, 1).  x ~ N(0, 1) rounded to the io dtype."""
+    base: DecodeSetup
+    conv_w: np.ndarray
+    conv_state0: np.ndarray
+
+    @property
+    def C(self) -> int:
+        b = self.base
+        return 2 * b.HK * b.Dk + b.HV * b.Dv
+
+    def step(self, s: int):
+        b = self.base
+        x = _store(_rng(b.seed, 200, s, 1).standard_normal((b.B, self.C), dtype=np.float32), b.io_dtype)
+        a = _rng(b.seed, 200, s, 4).standard_normal((b.B, b.HV), dtype=np.float32)
+        bb = _rng(b.seed, 200, s, 5).standard_normal((b.B, b.HV), dtype=np.float32)
+        return x, a, bb
+
+
+def decode_fused(B: int = 64, H: int = 32, D: int = 128, io_dtype: str = BF16, seed: int = 1,
+                 HK: int | None = None) -> FusedDecodeSetup:
+    base = decode(B=B, H=H, D=D, io_dtype=io_dtype, seed=seed, HK=HK)
+    C = 2 * base.HK * D + H * D
+    conv_w = (0.5 * _rng(seed, 200, 0, 7).standard_normal((C, 4), dtype=np.float32)).astype(np.float32)
+    conv_state0 = _rng(seed, 200, 0, 8).standard_normal((B, C, 3), dtype=np.float32)
+    return FusedDecodeSetup(base=base, conv_w=conv_w, conv_state0=conv_state0)

@@ -265,6 +265,32 @@ GDN_API gdn_status gdn_decode_step_gated(const void* q, const void* k, const voi
                            float scale, int32_t qk_l2norm, void* o, void* stream);
 
 /*
+ * gdn_decode_step_fused -- the whole decode step from raw projections in one kernel:
+ * the causal depthwise convolution of kernel 4 that the Qwen3-next page (section 3.1)
+ * places before the gated update (kernel size from the tutorial page, section 6,
+ * linear_conv_kernel_dim = 4), the q/k L2 norm, the gates and the state update.
+ *   x      [B, C] io_dtype, C = 2 HK Dk + HV Dv: per sequence the raw q | k | v
+ *          projections of the current token, q/k head-major then v head-major  (read)
+ *   conv_w [C, 4] fp32, taps oldest first: y = w0 x_{t-3} + w1 x_{t-2} + w2 x_{t-1} + w3 x_t
+ *   conv_state_in  [B, 3, C] fp32, the three previous inputs, oldest first      (read)
+ *   conv_state_out [B, 3, C] fp32, the three newest inputs after this token     (written;
+ *          must not overlap conv_state_in: value heads that share a q/k head read the
+ *          old q/k channels while another writes the new ones)
+ *   conv_act  0: q, k, v = y;  1: SiLU, y * sigmoid(y)  (the pages name no activation)
+ *   a, b, A_log, dt_bias, state, o and the rest as gdn_decode_step_gated.
+ * Dk = Dv = 128 only (others: UNSUPPORTED).  q, k, v are kept in fp32 after the
+ * convolution (no rounding to io_dtype).
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, ALIAS (any output over any input or another
+ * output), CUDA.
+ */
+GDN_API gdn_status gdn_decode_step_fused(const void* x, gdn_dtype io_dtype,
+                           const float* conv_w, const float* conv_state_in, float* conv_state_out,
+                           int32_t conv_act, const void* a, const void* b, gdn_dtype ab_dtype,
+                           const float* A_log, const float* dt_bias, float* state,
+                           int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                           float scale, int32_t qk_l2norm, void* o, void* stream);
+
+/*
  * gdn_decode_status -- synchronises the current device and writes its decode error
  * word (GDN_DEVERR_NONE or GDN_DEVERR_TIMEOUT, shared by every decode launch on that
  * device) into *device_error, then clears it.  This is library bookkeeping with no

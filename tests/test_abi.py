@@ -157,6 +157,27 @@ def test_prefill_host_validation(L):
     assert call(a10=0) == 0                     # B = 0: nothing to do
 
 
+def test_decode_fused_validation(L):
+    f = L.gdn_decode_step_fused
+    # x, io, w, cs_in, cs_out, act, a, b, ab, A_log, dt_bias, state, B, HK, HV, Dk, Dv, scale, l2, o, stream
+    base = [A, 1, A + MB, A + 2 * MB, A + 3 * MB, 1, A + 4 * MB, A + 5 * MB, 0, A + 6 * MB, A + 7 * MB,
+            A + 16 * MB, 4, 2, 4, 128, 128, 1.0, 1, A + 9 * MB, None]
+    def call(**kw):
+        a = list(base)
+        for i, val in kw.items():
+            a[int(i[1:])] = val
+        return f(*a)
+    assert call(a0=None) == 1
+    assert call(a2=None) == 1
+    assert call(a5=2) == 4                      # activation code
+    assert call(a15=64) == 4                    # d = 128 only
+    assert call(a14=3) == 2                     # HV % HK
+    assert call(a3=A + 2 * MB + 4) == 3         # conv_state_in misaligned
+    assert call(a4=A + 2 * MB) == 5             # conv_state_out over conv_state_in
+    assert call(a19=A + 16 * MB) == 5           # o over the state
+    assert call(a12=0) == 0                     # B = 0: nothing to do
+
+
 def test_decode_status_null(L):
     assert L.gdn_decode_status(None) == 1
 
