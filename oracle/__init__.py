@@ -20,6 +20,9 @@ Public functions (all fp64 numpy in, fp64 numpy out):
 * ``decode_step(q, k, v, g, beta, state, ...) -> (o, new_state)`` -- the same
   recurrence for one token per sequence, the incremental update of the
   "QWEN3.5" Q&A page (question 2a).
+* ``out_gate(o, z, w, eps=1e-6) -> out`` -- the output epilogue: zero-centred
+  RMSNorm over the last axis (Qwen3-next page, section 3.2) times (1 + w), times a
+  sigmoid gate of z (the GDN resource-allocation page).
 * ``conv(x, w, state=None, act=0) -> (y, new_state)`` -- the causal depthwise
   convolution of kernel 4 that the Qwen3-next page (section 3.1) puts before the
   gated update, with its rolling state of the three previous inputs.
@@ -83,6 +86,8 @@ class OracleLib:
         lib.gdn_oracle_conv.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_int, _dp, _dp]
         lib.gdn_oracle_conv.restype = None
+        lib.gdn_oracle_out_gate.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, _dp]
+        lib.gdn_oracle_out_gate.restype = None
         lib.gdn_oracle_max_threads.argtypes = []
         lib.gdn_oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
@@ -152,6 +157,19 @@ class OracleLib:
             raise ValueError(f"gdn_oracle_recurrence failed with code {rc}")
         return o.reshape(out_shape), hT
 
+    # -- output epilogue ---------------------------------------------------
+    def out_gate(self, o, z, w, eps: float = 1e-6):
+        """o, z [..., D]; w [D].  Returns o * rsqrt(mean(o^2) + eps) * (1 + w) * sigmoid(z)."""
+        o = _f64(o)
+        z = _f64(z)
+        w = _f64(w)
+        D = o.shape[-1]
+        if z.shape != o.shape or w.shape != (D,):
+            raise ValueError("out_gate: o, z must share a shape [..., D]; w must be [D]")
+        out = np.empty_like(o)
+        self.lib.gdn_oracle_out_gate(_ptr(o), _ptr(z), _ptr(w), o.size // D, D, float(eps), _ptr(out))
+        return out
+
     # -- convolution prologue --------------------------------------------
     def conv(self, x, w, state=None, act: int = 0):
         """x [B, T, C]; w [C, 4] (taps oldest first); state [B, C, 3] or None.
@@ -200,6 +218,10 @@ def recurrence(q, k, v, g, beta, h0=None, cu_seqlens=None, scale=1.0,
                l2norm=True, threads=0):
     return default().recurrence(q, k, v, g, beta, h0=h0, cu_seqlens=cu_seqlens,
                                 scale=scale, l2norm=l2norm, threads=threads)
+
+
+def out_gate(o, z, w, eps=1e-6):
+    return default().out_gate(o, z, w, eps=eps)
 
 
 def conv(x, w, state=None, act=0):

@@ -42,6 +42,14 @@
  *   name no activation, so act is the identity or, on request, SiLU
  *   (x * sigmoid(x)).
  *
+ *   Output epilogue (the Qwen3-next page, section 3.2, gives the zero-centred RMSNorm:
+ *   x * rsqrt(mean(x^2) + eps) with a weight initialised to zero, so the scale is
+ *   1 + weight; the GDN resource-allocation page says the output gate is usually a
+ *   sigmoid applied to the attention output before the residual add):
+ *       out = o * rsqrt(mean_j o_j^2 + eps) * (1 + w) * sigmoid(z)
+ *   per (token, value head) over the Dv values.  Readings: eps = 1e-6; z is the gate's
+ *   input, given per element; w is shared by the value heads.
+ *
  * Everything is fp64.  No blocking, chunking or reordering: one token at a
  * time, exactly the formula above.  OpenMP only splits independent
  * (sequence, value head) pairs across threads.
@@ -201,6 +209,21 @@ void gdn_oracle_conv(const double* x, const double* w, const double* state_in,
             }
             for (int i = 0; i < 3; ++i) state_out[(b * C + c) * 3 + i] = win[i];
         }
+    }
+}
+
+/* Zero-centred RMSNorm and sigmoid gate of rows of length D.  o, z: [rows, D];
+ * w: [D]; out: [rows, D]. */
+void gdn_oracle_out_gate(const double* o, const double* z, const double* w, int64_t rows, int64_t D,
+                         double eps, double* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* x = o + r * D;
+        double ss = 0.0;
+        for (int64_t j = 0; j < D; ++j) ss += x[j] * x[j];
+        const double inv = 1.0 / sqrt(ss / (double)D + eps);
+        for (int64_t j = 0; j < D; ++j)
+            out[r * D + j] = x[j] * inv * (1.0 + w[j]) * oracle_sigmoid(z[r * D + j]);
     }
 }
 

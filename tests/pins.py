@@ -15,6 +15,8 @@ rests on; none re-types the oracle's loop:
 * a brute-force expanded product of the per-token transition matrices;
 * structural facts: linearity in (v, S0), contraction bound, independence of
   packed sequences, grouped-head mapping, state carry, the chunked algebra;
+* the output epilogue: a hand-worked example (``golden/out_gate_hand.json``), scale
+  invariance, unit RMS of the plain norm, the gate against scipy, the place of eps;
 * the convolution prologue: a hand-worked example (``golden/conv_hand.json``),
   the impulse response, the state as the three past inputs, state carry,
   linearity, and SiLU against scipy's logistic function.
@@ -446,6 +448,45 @@ def pin_conv_linear_and_silu(orc):
     np.testing.assert_allclose(ys, y1 * expit(y1), rtol=1e-14, atol=1e-15)
 
 
+# ---------------------------------------------------------------------------
+# the output epilogue (Qwen3-next page, section 3.2; GDN resource-allocation page)
+# ---------------------------------------------------------------------------
+def pin_out_gate_hand(orc):
+    """A two-value row worked by hand."""
+    d = json.load(open(os.path.join(GOLDEN, "out_gate_hand.json")))
+    out = orc.out_gate(np.array([d["o"]]), np.array([d["z"]]), np.array(d["w"]), eps=d["eps"])
+    np.testing.assert_allclose(out[0], np.array(d["out"]), rtol=1e-15)
+
+
+def pin_out_gate_properties(orc):
+    """With eps = 0: scaling o by c > 0 changes nothing; with w = 0 and an open gate the
+    row has unit RMS (the plain RMSNorm); the gate multiplies by scipy's logistic
+    sigmoid of z; the sign of each element is that of o."""
+    from scipy.special import expit
+    rng = _rng(65)
+    rows, D = 5, 16
+    o = rng.standard_normal((rows, D))
+    z = rng.standard_normal((rows, D))
+    w = 0.3 * rng.standard_normal(D)
+    out = orc.out_gate(o, z, w, eps=0.0)
+    np.testing.assert_allclose(orc.out_gate(7.5 * o, z, w, eps=0.0), out, rtol=1e-13)
+    plain = orc.out_gate(o, np.full_like(z, 40.0), np.zeros(D), eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(plain ** 2, axis=-1)), np.ones(rows), rtol=1e-12)
+    gated0 = orc.out_gate(o, np.full_like(z, 40.0), w, eps=0.0)
+    np.testing.assert_allclose(out, gated0 * expit(z) / expit(40.0), rtol=1e-13)
+    assert np.all(np.sign(out) == np.sign(o))
+
+
+def pin_out_gate_eps(orc):
+    """eps sits inside the square root with the mean: a zero row stays zero, and a row of
+    RMS s gets the factor 1 / sqrt(s^2 + eps)."""
+    D = 8
+    o = np.full((1, D), 1e-3)
+    out = orc.out_gate(o, np.full((1, D), 40.0), np.zeros(D), eps=1e-6)
+    np.testing.assert_allclose(out, o / np.sqrt(1e-6 + 1e-6), rtol=1e-12)
+    assert np.all(orc.out_gate(np.zeros((1, D)), np.zeros((1, D)), np.zeros(D)) == 0.0)
+
+
 ALL_PINS = [
     pin_gates_library, pin_gates_hand, pin_gates_dt_construction, pin_hand_worked,
     pin_no_write_keeps_state, pin_orthonormal_retrieval, pin_full_write_any_decay,
@@ -453,5 +494,5 @@ ALL_PINS = [
     pin_contraction_bound, pin_packed_sequences_independent, pin_grouped_heads, pin_l2norm,
     pin_state_carry, pin_chunked_algebra,
     pin_conv_hand, pin_conv_impulse_response, pin_conv_state_is_past_input, pin_conv_state_carry,
-    pin_conv_linear_and_silu,
+    pin_conv_linear_and_silu, pin_out_gate_hand, pin_out_gate_properties, pin_out_gate_eps,
 ]

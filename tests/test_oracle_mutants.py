@@ -33,6 +33,10 @@ MUTANTS = {
     "conv_taps_reversed": ("acc += w[c * 4 + i] * win[i];", "acc += w[c * 4 + 3 - i] * win[i];"),
     "conv_state_not_shifted": ("win[1] = win[2];", "win[1] = win[3];"),
     "conv_silu_sign": ("acc * oracle_sigmoid(acc)", "acc * oracle_sigmoid(-acc)"),
+    "norm_eps_outside": ("1.0 / sqrt(ss / (double)D + eps)", "1.0 / (sqrt(ss / (double)D) + eps)"),
+    "norm_sum_not_mean": ("1.0 / sqrt(ss / (double)D + eps)", "1.0 / sqrt(ss + eps)"),
+    "norm_weight_not_centred": ("* (1.0 + w[j]) *", "* w[j] *"),
+    "gate_sign": ("oracle_sigmoid(z[r * D + j])", "oracle_sigmoid(-z[r * D + j])"),
 }
 
 _CHILD = r"""
