@@ -46,6 +46,9 @@ _SIGS = {
     "gdn_chunk_prefill": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                            _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "gdn_chunk_prefill_status": ([_vp, _vp, ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_chunk_prefill_outgate": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+                                   _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp],
+                                  ctypes.c_int),
     "gdn_decode_step": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                          _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
@@ -162,7 +165,7 @@ def prefill_workspace_bytes(n_tokens, n_seqs, HK, HV, Dk, Dv, BT, io_dtype) -> i
 
 def gdn_chunk_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, BT: int = 64,
                       scale: float = 1.0, qk_l2norm: bool = True, output_final_state: bool = True,
-                      o=None, final_state=None, workspace=None):
+                      o=None, final_state=None, workspace=None, outgate=None):
     """Chunked prefill.  Dense: q, k [B, T, HK, Dk], v [B, T, HV, Dv], g, beta [B, T, HV].
     Packed: B = 1 and cu_seqlens int32 [N + 1].  Returns (o, final_state or None)."""
     B, T, HK, Dk = q.shape
@@ -189,12 +192,30 @@ def gdn_chunk_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, BT:
         _check(4, "gdn_chunk_prefill")
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    st = lib().gdn_chunk_prefill(
-        _ptr(q), _ptr(k), _ptr(v), dcode, _ptr(g), _ptr(beta), _ptr(initial_state),
-        _ptr(cu_seqlens), B, T, N, HK, HV, Dk, Dv, BT, float(scale), int(bool(qk_l2norm)),
-        _ptr(o), _ptr(final_state), _ptr(workspace), workspace.numel(), _stream())
-    _check(st, "gdn_chunk_prefill")
+    if outgate is None:
+        st = lib().gdn_chunk_prefill(
+            _ptr(q), _ptr(k), _ptr(v), dcode, _ptr(g), _ptr(beta), _ptr(initial_state),
+            _ptr(cu_seqlens), B, T, N, HK, HV, Dk, Dv, BT, float(scale), int(bool(qk_l2norm)),
+            _ptr(o), _ptr(final_state), _ptr(workspace), workspace.numel(), _stream())
+        _check(st, "gdn_chunk_prefill")
+    else:
+        z, norm_w, eps = outgate
+        if z.shape != o.shape or z.dtype != q.dtype or norm_w.shape != (Dv,) or norm_w.dtype != torch.float32:
+            raise ValueError("z must be shaped and typed like o; norm_w fp32 [Dv]")
+        st = lib().gdn_chunk_prefill_outgate(
+            _ptr(q), _ptr(k), _ptr(v), dcode, _ptr(g), _ptr(beta), _ptr(initial_state),
+            _ptr(cu_seqlens), B, T, N, HK, HV, Dk, Dv, BT, float(scale), int(bool(qk_l2norm)),
+            _ptr(z), _ptr(norm_w), float(eps), _ptr(o), _ptr(final_state), _ptr(workspace), workspace.numel(),
+            _stream())
+        _check(st, "gdn_chunk_prefill_outgate")
     return o, final_state
+
+
+def gdn_chunk_prefill_outgate(q, k, v, g, beta, z, norm_w, eps: float = 1e-6, **kw):
+    """gdn_chunk_prefill with the output epilogue: each output row of a value head becomes
+    o * rsqrt(mean(o^2) + eps) * (1 + norm_w) * sigmoid(z); z like o, norm_w fp32 [Dv].
+    Keyword arguments as gdn_chunk_prefill."""
+    return gdn_chunk_prefill(q, k, v, g, beta, outgate=(z, norm_w, eps), **kw)
 
 
 def gdn_chunk_prefill_status(workspace: torch.Tensor) -> int:

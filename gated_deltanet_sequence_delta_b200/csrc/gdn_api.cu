@@ -98,12 +98,15 @@ size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seqs, int32
     return gdn::kStatusBytes;
 }
 
-gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
-                             const float* g, const float* beta, const float* initial_state,
-                             const int32_t* cu_seqlens, int32_t B, int64_t T, int32_t n_seqs,
-                             int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
-                             float scale, int32_t qk_l2norm, void* o, float* final_state,
-                             void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// gdn_chunk_prefill, with the output epilogue when z is given (tensor-core path only)
+gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype io_dtype, const float* g,
+                        const float* beta, const float* initial_state, const int32_t* cu_seqlens, int32_t B,
+                        int64_t T, int32_t n_seqs, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
+                        float scale, int32_t qk_l2norm, const void* z, const float* norm_w, float eps, void* o,
+                        float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
     // ---- sizes -----------------------------------------------------------------
     if (B < 0 || T < 0 || n_seqs < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || BT <= 0)
         return GDN_ERR_SHAPE;
@@ -124,8 +127,10 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dt
     if (!workspace) return GDN_ERR_WORKSPACE;
     if (workspace_bytes < need) return GDN_ERR_WORKSPACE;
     if (n_tok > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
+    if (z && (!norm_w || !(eps >= 0.f))) return norm_w ? GDN_ERR_SHAPE : GDN_ERR_NULL;
+    if (z && !(io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT))) return GDN_ERR_UNSUPPORTED;
     if (cu_seqlens == nullptr && n_tok == 0 && final_state == nullptr) return GDN_OK;
-    const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, workspace};
+    const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, workspace, z, norm_w};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     // ---- aliasing ----------------------------------------------------------------
@@ -137,8 +142,9 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dt
     const Range rh0{initial_state, state_bytes}, rcu{cu_seqlens, cu_seqlens ? (size_t)(n_seqs + 1) * 4 : 0};
     const Range ro{o, (size_t)n_tok * HV * Dv * es}, rhT{final_state, state_bytes};
     const Range rws{workspace, workspace_bytes};
+    const Range rz{z, z ? (size_t)n_tok * HV * Dv * es : 0}, rnw{norm_w, z ? (size_t)Dv * 4 : 0};
     for (Range out : {ro, rhT, rws}) {
-        for (Range in : {rq, rk, rv, rg, rb, rcu})
+        for (Range in : {rq, rk, rv, rg, rb, rcu, rz, rnw})
             if (overlap(out, in)) return GDN_ERR_ALIAS;
     }
     if (overlap(ro, rhT) || overlap(ro, rws) || overlap(rhT, rws) || overlap(ro, rh0) ||
@@ -160,11 +166,36 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dt
     a.g = g; a.beta = beta; a.h0 = initial_state; a.cu = cu_seqlens;
     a.T = T; a.n_seqs = n_seqs; a.HK = HK; a.HV = HV; a.Dk = Dk; a.Dv = Dv; a.BT = BT;
     a.scale = scale; a.l2norm = qk_l2norm ? 1 : 0; a.o = o; a.hT = final_state;
+    a.z = z; a.norm_w = norm_w; a.eps = eps;
     a.status = status;
     a.scratch = static_cast<char*>(workspace) + gdn::kStatusBytes;
     a.scratch_bytes = workspace_bytes - gdn::kStatusBytes;
     if (use_tc) return cuda_status(gdn::launch_prefill_tc(a, workspace, s));
     return cuda_status(gdn::launch_prefill_cudacore(a, s));
+}
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                             const float* g, const float* beta, const float* initial_state,
+                             const int32_t* cu_seqlens, int32_t B, int64_t T, int32_t n_seqs,
+                             int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
+                             float scale, int32_t qk_l2norm, void* o, float* final_state,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT,
+                        scale, qk_l2norm, nullptr, nullptr, 0.f, o, final_state, workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_chunk_prefill_outgate(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                                     const float* g, const float* beta, const float* initial_state,
+                                     const int32_t* cu_seqlens, int32_t B, int64_t T, int32_t n_seqs,
+                                     int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT, float scale,
+                                     int32_t qk_l2norm, const void* z, const float* norm_w, float eps, void* o,
+                                     float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!z) return GDN_ERR_NULL;
+    return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT,
+                        scale, qk_l2norm, z, norm_w, eps, o, final_state, workspace, workspace_bytes, stream);
 }
 
 gdn_status gdn_chunk_prefill_status(const void* workspace, void* stream, int32_t* device_error) {

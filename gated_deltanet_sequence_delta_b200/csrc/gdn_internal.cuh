@@ -115,6 +115,9 @@ struct PrefillArgs {
     int l2norm;
     void* o;
     float* hT;                // may be null
+    const void* z;            // output epilogue gate inputs [.., HV, Dv] io dtype, or null (none)
+    const float* norm_w;      // output epilogue norm weights [Dv] (with z)
+    float eps;                // output epilogue norm epsilon (with z)
     int32_t* status;          // device status word (workspace)
     void* scratch;            // workspace after the status words
     size_t scratch_bytes;

@@ -66,6 +66,11 @@ __device__ __forceinline__ float pow2_above(float max_abs) {
     return ldexpf(1.f, e);
 }
 
+// sigmoid(x) = 1 / (1 + exp(-x)) from the fast exponential and the approximate divide; both
+// are within a few ulp of fp32, far below the bf16 rounding of the output, and the limits
+// come out right (exp(-x) = inf gives 0, exp(-x) = 0 gives 1)
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -634,7 +639,13 @@ struct CarrySmem {
     f16 Dl[C * NS];        // scaled Delta, same layout (K = tokens)
     f16 Dt[C * NS];        // scaled Delta~ = diag(exp(G_C - G)) Delta
     float red[4];
-    uint64_t full[NSTAGE], empty[NSTAGE], bar_a, bar_b, bar_o, h0_ready, d_ready;
+    // output epilogue: per chunk parity, this CTA's per-row sums of squares and those
+    // received from the other slices; the norm weights of this slice
+    float oloc[2][C];
+    float opart[2][D / NS][C];
+    float onw[NS];   // 1 + w of this slice's values
+    // bar_o: one per output buffer, so that a deferred wait can never fall two phases behind
+    uint64_t full[NSTAGE], empty[NSTAGE], bar_a, bar_b, bar_o[3], h0_ready, d_ready, obar[2];
     uint32_t tmem_base;
     volatile int abort;
 };
@@ -671,9 +682,9 @@ __device__ __forceinline__ void store_op_row(f16* op, int k, const float* v, flo
 }
 
 // Per chunk c, the MMA warp issues (each group committed to its own mbarrier):
-//   a: [W; Q_hat] H0     (M=128, 8 MMAs)  -> D_a[c & 1]  rows 0-63 W H0, rows 64-127 Q_hat H0
-//   b: K_hat^T Delta~    (M=128, 4 MMAs)  -> D_b         state update
-//   c: [0; P] Delta      (M=128, 4 MMAs)  -> D_c[c & 1]  rows 64-127 P Delta
+//   a: [W; Q_hat] H0     (M=128, 8 MMAs)  -> D_a[c % nb]  rows 0-63 W H0, rows 64-127 Q_hat H0
+//   b: K_hat^T Delta~    (M=128, 4 MMAs)  -> D_b          state update
+//   c: [0; P] Delta      (M=128, 4 MMAs)  -> D_c[c % nb]  rows 64-127 P Delta
 // Epilogue threads 0-63 turn D_a rows into Delta, Delta~; all 128 update the state rows
 // from D_b; threads 64-127 write the output rows of chunk c while chunk c+1's MMAs run.
 // The two sides meet only through mbarriers (h0_ready, d_ready: one arrival per epilogue
@@ -681,13 +692,24 @@ __device__ __forceinline__ void store_op_row(f16* op, int k, const float* v, flo
 // arrive on d_ready as soon as they have read the chunk's scalars, then
 // write the previous chunk's output rows while Delta and the state MMA proceed; the
 // stage is released only after every thread's reads of it).
+//
+// OUTG adds the output epilogue out = o rsqrt(mean(o^2) + eps) (1 + w) sigmoid(z) over the
+// 128 values of a head, which live in the head's four slice CTAs: those run as one
+// thread-block cluster (cluster rank = slice), and each output row's four partial sums of
+// squares cross over distributed shared memory, announced by remote mbarrier arrivals.
+// To keep that exchange off the serial chain the output warps write chunk c-2 (not c-1)
+// while chunk c's Delta and state MMA run, so D_a and D_c rotate over three buffers
+// (nb = 3) instead of two.
+template <bool OUTG>
 __global__ void __launch_bounds__(kCarryThreads, 1)
 chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qk,
                    const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_u,
                    const float* __restrict__ SCg, const int32_t* __restrict__ cu,
                    const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HK, int HV,
                    const float* __restrict__ h0, float* __restrict__ hT, bf16* __restrict__ o,
+                   const bf16* __restrict__ zg, const float* __restrict__ norm_w, float eps,
                    int32_t* __restrict__ status) {
+    constexpr int nb = OUTG ? 3 : 2;   // buffers of D_a and D_c
     extern __shared__ uint8_t smem_raw[];
     CarrySmem& S = *reinterpret_cast<CarrySmem*>(align1024(smem_raw));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -697,11 +719,14 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
     const int h = idx % HV;       idx /= HV;
     const int n = idx;
     const int hk = h / (HV / HK);
-    if (*reinterpret_cast<volatile int32_t*>(status) != 0) return;
+    // Without clusters a CTA may leave at once; with them every CTA must reach both cluster
+    // barriers, so a failed earlier stage only empties the work.
+    const bool failed = *reinterpret_cast<volatile int32_t*>(status) != 0;
+    if (!OUTG && failed) return;
     const int64_t bos = cu ? (int64_t)cu[n] : (int64_t)n * T;
     const int64_t len = cu ? (int64_t)cu[n + 1] - cu[n] : T;
     const int c0 = chunk_off[n];
-    const int nch = chunk_off[n + 1] - c0;
+    const int nch = failed ? 0 : chunk_off[n + 1] - c0;
 
     if (warp == 0) {
         tc::tmem_alloc(&S.tmem_base, kCarryTmemCols);
@@ -714,12 +739,17 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         }
         tc::mbar_init(&S.bar_a, 1);
         tc::mbar_init(&S.bar_b, 1);
-        tc::mbar_init(&S.bar_o, 1);
+        for (int i = 0; i < 3; ++i) tc::mbar_init(&S.bar_o[i], 1);
         tc::mbar_init(&S.h0_ready, 4);   // one arrival per epilogue warp
         tc::mbar_init(&S.d_ready, 4);
+        if (OUTG) {   // one local arrival per use, plus the peers' bulk copies as transactions
+            tc::mbar_init(&S.obar[0], 1);
+            tc::mbar_init(&S.obar[1], 1);
+        }
         tc::fence_mbar_init();
         S.abort = 0;
     }
+    if (OUTG && tid < NS) S.onw[tid] = 1.f + norm_w[vs * NS + tid];   // the (1 + w) factor
     // zero rows 0-63 of the P operands (the producer only ever writes rows 64-127)
     for (int e = tid; e < NSTAGE * 64 * 64 / 8; e += kCarryThreads) {
         const int st = e / (64 * 64 / 8), r = e % (64 * 64 / 8);
@@ -728,9 +758,10 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
     tc::fence_async_smem();
     tc::tc_fence_before();
     __syncthreads();
+    if (OUTG) tc::cluster_sync();   // every slice CTA's barriers exist before any remote arrival
     tc::tc_fence_after();
     const uint32_t tmem = S.tmem_base;
-    const uint32_t tA = tmem, tB = tmem + 64, tC = tmem + 96;   // tA, tC: +32 per chunk parity
+    const uint32_t tA = tmem, tB = tmem + nb * 32, tC = tmem + nb * 32 + 32;   // tA, tC: +32 per buffer
 
     if (warp == 4) {
         // ---------------- producer: stream the chunks through the ring ----------------
@@ -776,7 +807,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                     break;
                 }
                 tc::tc_fence_after();
-                const uint32_t par = (uint32_t)(c & 1) * 32;
+                const uint32_t par = (uint32_t)(c % nb) * 32;
                 // descriptors built once; a k-step only advances the start-address field
                 const uint64_t da = tc::desc_sw128(tc::smem_u32(&B.A[0][0]), 16, 1024);
                 const uint64_t dh = desc_noswz(tc::smem_u32(S.H0[c & 1]), kOpLBO, kOpSBO);
@@ -802,7 +833,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tC + par, dp + (uint64_t)((kk * 32) >> 4), ddl + (uint64_t)((kk * 2 * kOpLBO) >> 4),
                                  idA, kk > 0);
-                tc::mma_commit(&S.bar_o);
+                tc::mma_commit(&S.bar_o[c % nb]);
                 tc::mma_commit(&S.empty[st]);   // the stage's operands are consumed
             }
         }
@@ -831,9 +862,85 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&S.h0_ready);
         bool ok = true;
-        float a_prev = 0.f;
-        int cn_prev = 0;
-        int64_t tok_prev = 0;
+        float a_prev = 0.f;          // per-row scalar, length and first token of the chunk whose
+        int cn_prev = 0;             //   output is written next (plain: the previous chunk;
+        int64_t tok_prev = 0;        //   OUTG: two chunks back, its successor in the *_nxt copies)
+        float a_nxt = 0.f;
+        int cn_nxt = 0;
+        int64_t tok_nxt = 0;
+        // OUTG: the gate inputs z of this row's values for the next chunk whose output is
+        // written, loaded one output call ahead so that their latency is off the chain
+        uint4 zpre[NS / 8];
+        auto load_z = [&](int64_t tok0, int rows) {
+            const int i = t - 64;
+            if (OUTG && i < rows) {
+                const uint4* zr = reinterpret_cast<const uint4*>(zg + ((tok0 + i) * HV + h) * D + vs * NS);
+#pragma unroll
+                for (int qq = 0; qq < NS / 8; ++qq) zpre[qq] = zr[qq];
+            }
+        };
+        // output rows of chunk cc (threads 64-127, row t - 64), from D_a and D_c buffer cc % nb;
+        // OUTG with pre set then starts the z loads of the chunk held in the *_nxt copies
+        auto write_output = [&](int cc, bool pre) -> bool {
+            const int i = t - 64;
+            bool good = tc::mbar_wait(&S.bar_o[cc % nb], (uint32_t)((cc / nb) & 1));
+            tc::tc_fence_after();
+            const uint32_t par = (uint32_t)(cc % nb) * 32;
+            float q[NS], z[NS];
+            tc::tmem_ld32(tA + par + lane_base, q);
+            tc::tmem_ld32(tC + par + lane_base, z);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < NS; ++j) q[j] = fmaf(a_prev, q[j], z[j]) * inv_sc;   // the core output
+            if (OUTG) {
+                // this slice's sum of squares per row; the 64 rows go to each other slice CTA of
+                // the head in one bulk copy, which completes on that CTA's barrier
+                float ps = 0.f;
+#pragma unroll
+                for (int j = 0; j < NS; ++j) ps = fmaf(q[j], q[j], ps);
+                const int p = cc & 1;
+                S.oloc[p][i] = ps;
+                tc::fence_async_smem();
+                tc::named_bar(2, 64);   // the output warps' 64 rows are in oloc
+                if (t == 64) {
+                    tc::mbar_expect_tx(&S.obar[p], (nslices - 1) * C * 4);
+#pragma unroll
+                    for (int rk = 0; rk < nslices; ++rk)
+                        if (rk != vs)
+                            tc::bulk_copy_to_peer(tc::cluster_map(tc::smem_u32(&S.opart[p][vs][0]), rk), S.oloc[p], C * 4,
+                                                  tc::cluster_map(tc::smem_u32(&S.obar[p]), rk));
+                }
+                good = tc::mbar_wait_cluster(&S.obar[p], (uint32_t)((cc >> 1) & 1)) && good;
+                float ss = ps;
+#pragma unroll
+                for (int rk = 0; rk < nslices; ++rk)
+                    if (rk != vs) ss += S.opart[p][rk][i];
+                const float inv_rms = rsqrtf(ss * (1.f / D) + eps);
+                if (i < cn_prev) {
+#pragma unroll
+                    for (int qq = 0; qq < NS / 8; ++qq) {
+                        const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&zpre[qq]);
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const float2 zz = __bfloat1622float2(e[e2]);
+                            const int j = qq * 8 + e2 * 2;
+                            q[j] = q[j] * inv_rms * S.onw[j] * sigmoid_fast(zz.x);
+                            q[j + 1] = q[j + 1] * inv_rms * S.onw[j + 1] * sigmoid_fast(zz.y);
+                        }
+                    }
+                }
+                if (pre) load_z(tok_nxt, cn_nxt);
+            }
+            if (i < cn_prev) {
+                __align__(16) bf16 ob[NS];
+#pragma unroll
+                for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(q[j]);
+                uint4* dst = reinterpret_cast<uint4*>(o + ((tok_prev + i) * HV + h) * D + vs * NS);
+#pragma unroll
+                for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
+            }
+            return good;
+        };
         for (int c = 0; c < nch && ok; ++c) {
             const int st = c % NSTAGE, rr = c / NSTAGE;
             const CarryStage& B = S.st[st];
@@ -842,22 +949,23 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
             const int cn = (int)(rem < C ? rem : C);
             ok = tc::mbar_wait(&S.full[st], rr & 1);
             const float gC = B.SC[SC_GC];
+            float a_cur = 0.f;
             if (warp < 2) {
                 // ---- Delta rows (threads 0-63) ----------------------------------------------
                 ok = tc::mbar_wait(&S.bar_a, c & 1) && ok;
                 tc::tc_fence_after();
                 float x[NS];
-                tc::tmem_ld32(tA + (uint32_t)(c & 1) * 32 + lane_base, x);
+                tc::tmem_ld32(tA + (uint32_t)(c % nb) * 32 + lane_base, x);
                 tc::tmem_wait_ld();
                 const float dr = B.SC[64 + t], uinv = B.SC[SC_UINV];
                 const uint4* urow = reinterpret_cast<const uint4*>(B.U + t * NS);
                 float dv[NS];
 #pragma unroll
-                for (int nb = 0; nb < NS / 8; ++nb) {   // 16-byte pieces of the row
-                    const uint4 u = urow[nb];
+                for (int nb8 = 0; nb8 < NS / 8; ++nb8) {   // 16-byte pieces of the row
+                    const uint4 u = urow[nb8];
                     const f16* e = reinterpret_cast<const f16*>(&u);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) dv[nb * 8 + q] = __half2float(e[q]) * uinv;
+                    for (int q = 0; q < 8; ++q) dv[nb8 * 8 + q] = __half2float(e[q]) * uinv;
                 }
 #pragma unroll
                 for (int j = 0; j < NS; ++j) dv[j] -= x[j] * inv_sc;
@@ -868,32 +976,29 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&S.d_ready);
             } else {
-                // ---- output rows of the previous chunk (threads 64-127), under this chunk's
-                //      Delta epilogue and state MMA -------------------------------------------
-                const float a_cur = B.SC[t - 64];
+                // ---- output warps: the chunk's scalars, then the output rows of an earlier
+                //      chunk under this chunk's Delta epilogue and state MMA: plain, chunk
+                //      c - 1; OUTG, chunk c - 2, so that its cluster exchange has a whole chunk
+                //      of slack (D_a, D_c of chunk c - 2 live until chunk c + 1's MMAs) ----------
+                a_cur = B.SC[t - 64];
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&S.d_ready);   // the stage's scalars are read
-                if (c > 0) {
-                    ok = tc::mbar_wait(&S.bar_o, (c - 1) & 1) && ok;
-                    tc::tc_fence_after();
-                    const uint32_t par = (uint32_t)((c - 1) & 1) * 32;
-                    float q[NS], z[NS];
-                    tc::tmem_ld32(tA + par + lane_base, q);
-                    tc::tmem_ld32(tC + par + lane_base, z);
-                    tc::tmem_wait_ld();
-                    if (t - 64 < cn_prev) {
-                        __align__(16) bf16 ob[NS];
-#pragma unroll
-                        for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(a_prev, q[j], z[j]) * inv_sc);
-                        uint4* dst = reinterpret_cast<uint4*>(o + ((tok_prev + t - 64) * HV + h) * D + vs * NS);
-#pragma unroll
-                        for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
-                    }
+                if (!OUTG) {
+                    if (c > 0) ok = write_output(c - 1, false) && ok;
+                    a_prev = a_cur;
+                    cn_prev = cn;
+                    tok_prev = tok;
+                } else {
+                    if (c > 1) ok = write_output(c - 2, true) && ok;
+                    else if (c == 1) load_z(tok_nxt, cn_nxt);   // chunk 0's
+                    a_prev = a_nxt;
+                    cn_prev = cn_nxt;
+                    tok_prev = tok_nxt;
+                    a_nxt = a_cur;
+                    cn_nxt = cn;
+                    tok_nxt = tok;
                 }
-                a_prev = a_cur;
             }
-            cn_prev = cn;
-            tok_prev = tok;
             // ---- state rows (all 128) ---------------------------------------------------------
             ok = tc::mbar_wait(&S.bar_b, c & 1) && ok;
             tc::tc_fence_after();
@@ -911,22 +1016,21 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
             if (lane == 0) tc::mbar_arrive(&S.h0_ready);
             if (S.abort) ok = false;
         }
-        if (ok && nch > 0 && warp >= 2) {   // output rows of the last chunk
-            ok = tc::mbar_wait(&S.bar_o, (nch - 1) & 1);
-            tc::tc_fence_after();
-            const uint32_t par = (uint32_t)((nch - 1) & 1) * 32;
-            float q[NS], z[NS];
-            tc::tmem_ld32(tA + par + lane_base, q);
-            tc::tmem_ld32(tC + par + lane_base, z);
-            tc::tmem_wait_ld();
-            if (ok && t - 64 < cn_prev) {
-                __align__(16) bf16 ob[NS];
-#pragma unroll
-                for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(a_prev, q[j], z[j]) * inv_sc);
-                uint4* dst = reinterpret_cast<uint4*>(o + ((tok_prev + t - 64) * HV + h) * D + vs * NS);
-#pragma unroll
-                for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
+        if (warp >= 2) {   // output rows of the chunks still pending
+            if (OUTG) {
+                if (ok && nch > 1) {
+                    ok = write_output(nch - 2, true);
+                    a_prev = a_nxt;
+                    cn_prev = cn_nxt;
+                    tok_prev = tok_nxt;
+                } else if (nch == 1) {
+                    load_z(tok_nxt, cn_nxt);
+                    a_prev = a_nxt;
+                    cn_prev = cn_nxt;
+                    tok_prev = tok_nxt;
+                }
             }
+            if (ok && nch > 0) ok = write_output(nch - 1, false);
         }
         if (!ok) {
             record_timeout(status);
@@ -943,6 +1047,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         for (int i = 0; i < NSTAGE; ++i) (void)tc::mbar_wait(&S.full[i], 0, 50000000ull);
     }
     __syncthreads();
+    if (OUTG) tc::cluster_sync();   // no CTA leaves while a peer may still write its shared memory
     if (warp == 0) tc::tmem_dealloc(tmem, kCarryTmemCols);
 }
 
@@ -1102,11 +1207,35 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
         if (e != cudaSuccess) return e;
         count_launch();
     }
-    e = cudaFuncSetAttribute(chunk_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCarrySmemBytes);
-    if (e != cudaSuccess) return e;
     const unsigned blocks = (unsigned)a.n_seqs * (unsigned)a.HV * (unsigned)(D / NS);
-    chunk_carry_kernel<<<blocks, kCarryThreads, kCarrySmemBytes, s>>>(tw, tqk, tp, tu, SC, a.cu, chunk_off, a.T, a.n_seqs,
-                                                          a.HK, a.HV, a.h0, a.hT, (bf16*)a.o, a.status);
+    if (!a.z) {
+        e = cudaFuncSetAttribute(chunk_carry_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kCarrySmemBytes);
+        if (e != cudaSuccess) return e;
+        chunk_carry_kernel<false><<<blocks, kCarryThreads, kCarrySmemBytes, s>>>(
+            tw, tqk, tp, tu, SC, a.cu, chunk_off, a.T, a.n_seqs, a.HK, a.HV, a.h0, a.hT, (bf16*)a.o, nullptr,
+            nullptr, 0.f, a.status);
+    } else {   // the head's four column slices as one cluster (output epilogue)
+        e = cudaFuncSetAttribute(chunk_carry_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kCarrySmemBytes);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(blocks);
+        cfg.blockDim = dim3(kCarryThreads);
+        cfg.dynamicSmemBytes = kCarrySmemBytes;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = D / NS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, chunk_carry_kernel<true>, tw, tqk, tp, tu, (const float*)SC, a.cu,
+                               (const int32_t*)chunk_off, a.T, a.n_seqs, a.HK, a.HV, a.h0, a.hT, (bf16*)a.o,
+                               (const bf16*)a.z, a.norm_w, a.eps, a.status);
+        if (e != cudaSuccess) return e;
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();

@@ -189,6 +189,14 @@ def make_prefill(B: int, T: int, HK: int, HV: int, Dk: int, Dv: int, *, io_dtype
     return inp
 
 
+def outgate_inputs(n_tokens: int, HV: int, Dv: int, io_dtype: str, seed: int):
+    """Gate inputs z [n_tokens, HV, Dv] ~ N(0, 1) in the io dtype and norm weights
+    w [Dv] ~ N(0, 0.3^2) fp32 for the output epilogue."""
+    z = _store(_rng(seed, 300, 1).standard_normal((n_tokens, HV, Dv), dtype=np.float32), io_dtype)
+    w = (0.3 * _rng(seed, 300, 2).standard_normal(Dv, dtype=np.float32)).astype(np.float32)
+    return z, w
+
+
 def varlen_lengths(seed: int, total: int = 65536, lo: int = 512, hi: int = 8192) -> np.ndarray:
     """Sequence lengths ~ U_int[lo, hi] until they sum to ``total`` (last one truncated)."""
     rng = _rng(seed, _STREAM["lens"])

@@ -152,6 +152,31 @@ GDN_API gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * gdn_chunk_prefill_outgate -- gdn_chunk_prefill with the output epilogue fused into the
+ * output store: each output row of a value head (Dv values) becomes
+ *     o * rsqrt(mean(o^2) + eps) * (1 + norm_w) * sigmoid(z)
+ * the zero-centred RMSNorm of the Qwen3-next page (section 3.2: weight initialised to
+ * zero) and the sigmoid output gate of the GDN resource-allocation page (applied after the
+ * attention output, before the residual add).
+ *   z       [B, T, HV, Dv] (or [T_total, HV, Dv] packed) io_dtype, the gate inputs  (read)
+ *   norm_w  [Dv] fp32, shared by the value heads                                    (read)
+ *   eps     >= 0 (the workloads' reading: 1e-6)
+ * Other arguments as gdn_chunk_prefill, whose workspace size applies.  Only the
+ * tensor-core configuration (bf16, Dk = Dv = 128, BT = 64, HV / HK in {1, 2}); others
+ * return UNSUPPORTED.  Errors: those of gdn_chunk_prefill, NULL (z or norm_w), SHAPE
+ * (eps < 0 or NaN), ALIAS (o, final_state or workspace over z or norm_w).
+ */
+GDN_API gdn_status gdn_chunk_prefill_outgate(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                             const float* g, const float* beta,
+                             const float* initial_state, const int32_t* cu_seqlens,
+                             int32_t B, int64_t T, int32_t n_seqs,
+                             int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                             int32_t BT, float scale, int32_t qk_l2norm,
+                             const void* z, const float* norm_w, float eps,
+                             void* o, float* final_state,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reads the device status word of a prefill
  * workspace into *device_error (GDN_DEVERR_*).  Returns GDN_ERR_DEVICE if it
  * is nonzero, GDN_ERR_CUDA if the synchronisation failed, else GDN_OK.

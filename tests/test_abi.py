@@ -68,6 +68,31 @@ def test_prefill_validation(L):
     assert _prefill(L, N=0, B=0) == 0                     # nothing to do: no launch
 
 
+def _prefill_outgate(L, **kw):
+    args = dict(q=A, k=A + 64 * MB, v=A + 128 * MB, io=1, g=A + 192 * MB, beta=A + 200 * MB,
+                h0=None, cu=None, B=1, T=128, N=1, HK=2, HV=4, Dk=128, Dv=128, BT=64, scale=1.0,
+                l2=1, z=A + 512 * MB, nw=A + 600 * MB, eps=1e-6, o=A + 256 * MB, hT=A + 384 * MB,
+                ws=A + 448 * MB, ws_bytes=1 << 20)
+    args.update(kw)
+    return L.gdn_chunk_prefill_outgate(args["q"], args["k"], args["v"], args["io"], args["g"], args["beta"],
+                                       args["h0"], args["cu"], args["B"], args["T"], args["N"], args["HK"],
+                                       args["HV"], args["Dk"], args["Dv"], args["BT"], args["scale"],
+                                       args["l2"], args["z"], args["nw"], args["eps"], args["o"], args["hT"],
+                                       args["ws"], args["ws_bytes"], None)
+
+
+def test_prefill_outgate_validation(L):
+    assert _prefill_outgate(L, z=None) == 1
+    assert _prefill_outgate(L, nw=None) == 1
+    assert _prefill_outgate(L, eps=-1.0) == 2
+    assert _prefill_outgate(L, eps=float("nan")) == 2
+    assert _prefill_outgate(L, io=0, BT=64) == 4          # fp32: no tensor-core path, no epilogue
+    assert _prefill_outgate(L, HV=6, HK=2) == 4            # GQA group 3
+    assert _prefill_outgate(L, z=A + 512 * MB + 4) == 3    # misaligned
+    assert _prefill_outgate(L, o=A + 512 * MB + 64) == 5   # o over z
+    assert _prefill_outgate(L, N=0, B=0) == 0              # nothing to do
+
+
 def test_prefill_workspace_query(L):
     assert L.gdn_chunk_prefill_workspace_bytes(32768, 1, 16, 32, 128, 128, 64, 1) >= 256
     assert L.gdn_chunk_prefill_workspace_bytes(256, 1, 2, 2, 64, 64, 64, 0) >= 256
