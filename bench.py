@@ -382,6 +382,28 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
     del hq, hk_, hv, ha, hb, hAl, hdtb, ho, hh, hws
+
+    # ---------------- the same prefill with the output epilogue fused ----------------
+    # out = o rsqrt(mean(o^2) + eps) (1 + w) sigmoid(z) per (token, value head), inside the
+    # state-carry kernel (gdn_chunk_prefill_outgate); reported beside the core path
+    z, w = I.outgate_inputs(T, HV, D, I.BF16, replica_seed(87, rank))
+    zd, wd = dev_t(z).view(1, T, HV, D), dev_t(w)
+
+    def gated_step():
+        G.gdn_chunk_prefill_outgate(q, k, v, g, beta, zd, wd, 1e-6, BT=BT, o=o, final_state=hT, workspace=ws)
+
+    for _ in range(3):
+        gated_step()
+    barrier()
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    g0.record()
+    for _ in range(args.steps):
+        gated_step()
+    g1.record()
+    barrier()
+    gated_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
+    del zd, wd
     flops = prefill_flops_per_token(HK, HV, D, BT) * T
     pbytes = prefill_bytes_per_token(HK, HV, D) * T + HV * D * D * 4
     tflops = flops / (kernel_ms * 1e-3) / 1e12
@@ -403,6 +425,10 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "path": f"gdn_chunk_prefill_host, pinned host buffers, {E2E_PIECE}-token pieces"},
         "gpu_launches": launches,
+        "gated_output": {"what": "gdn_chunk_prefill_outgate: the same prefill with the gated RMSNorm output "
+                                 "epilogue (eps 1e-6) fused into the state carry; gates precomputed",
+                         "ms_per_call": gated_ms, "tokens_per_s": whole_job_rate(world, T, gated_ms),
+                         "core_prefill_ms_per_call": kernel_ms},
     }
 
 

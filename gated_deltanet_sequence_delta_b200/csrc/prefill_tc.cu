@@ -66,10 +66,14 @@ __device__ __forceinline__ float pow2_above(float max_abs) {
     return ldexpf(1.f, e);
 }
 
-// sigmoid(x) = 1 / (1 + exp(-x)) from the fast exponential and the approximate divide; both
-// are within a few ulp of fp32, far below the bf16 rounding of the output, and the limits
-// come out right (exp(-x) = inf gives 0, exp(-x) = 0 gives 1)
-__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (one special-function op, about
+// 2^-11 relative error): an absolute gate error below 2^-12, under the bf16 rounding of the
+// output for gates above 1/8 and a negligible absolute error below; saturates to 0 and 1
+__device__ __forceinline__ float sigmoid_fast(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -632,27 +636,49 @@ struct CarryStage {
     f16 U[64 * NS];        // scaled U columns of this slice, row-major (4 KB)
     float SC[SC_FLOATS];   // a[64], d[64], gamma_C, U scale, max |v|
 };
+constexpr int NZ = 4;   // ring of gate-input tiles (output epilogue)
+struct ZSlot {
+    bf16 z[C * NS];    // z of the chunk's rows, this slice's values, row-major (4 KB)
+    float a[C];        // the chunk's per-row output scalars
+};
 struct CarrySmem {
     CarryStage st[NSTAGE];
     f16 H0[2][D * NS];     // scaled fp16 state slice: MN-major unswizzled B operand (K = Dk),
                            //   by chunk parity
     f16 Dl[C * NS];        // scaled Delta, same layout (K = tokens)
     f16 Dt[C * NS];        // scaled Delta~ = diag(exp(G_C - G)) Delta
+    ZSlot zr[NZ];          // output epilogue: z tiles and scalars, chunk c in slot c % NZ
     float red[4];
     // output epilogue: per chunk parity, this CTA's per-row sums of squares and those
-    // received from the other slices; the norm weights of this slice
-    float oloc[2][C];
-    float opart[2][D / NS][C];
+    // received from the other slices (bulk-copy source and target: 16-byte aligned)
+    alignas(16) float oloc[2][C];
+    alignas(16) float opart[2][D / NS][C];
     float onw[NS];   // 1 + w of this slice's values
-    // bar_o: one per output buffer, so that a deferred wait can never fall two phases behind
+    float inv_sc;    // the data scale, for the output warps
+    // bar_o: one per output buffer, so that a deferred wait can never fall two phases behind;
+    // ofree: the output warps are done with an output buffer; zfull / zempty: the z ring
     uint64_t full[NSTAGE], empty[NSTAGE], bar_a, bar_b, bar_o[3], h0_ready, d_ready, obar[2];
+    uint64_t ofree[3], zfull[NZ], zempty[NZ];
     uint32_t tmem_base;
     volatile int abort;
 };
 constexpr size_t kCarrySmemBytes = sizeof(CarrySmem) + 1024;
+// targets and sources of TMA and bulk copies sit on 16-byte (swizzled tiles: 1024-byte) boundaries
+static_assert(sizeof(CarryStage) % 1024 == 0 && offsetof(CarryStage, K) % 1024 == 0 &&
+                  offsetof(CarryStage, P) % 1024 == 0 && offsetof(CarryStage, U) % 16 == 0 &&
+                  offsetof(CarryStage, SC) % 16 == 0,
+              "carry stage layout");
+static_assert(offsetof(CarrySmem, zr) % 16 == 0 && sizeof(ZSlot) % 16 == 0 && offsetof(ZSlot, a) % 16 == 0 &&
+                  offsetof(CarrySmem, oloc) % 16 == 0 && offsetof(CarrySmem, opart) % 16 == 0 &&
+                  offsetof(CarrySmem, H0) % 16 == 0 && offsetof(CarrySmem, Dl) % 16 == 0 &&
+                  offsetof(CarrySmem, Dt) % 16 == 0,
+              "carry shared-memory layout");
 constexpr uint32_t kCarryTmemCols = 256;
 constexpr uint32_t kStageTxBytes = 2 * 128 * 64 * 2 + 2 * 64 * 64 * 2 + 64 * 64 * 2 + 64 * NS * 2 + SC_FLOATS * 4;
-constexpr int kCarryThreads = 192;   // warps 0-3 epilogues, warp 4 TMA producer, warp 5 MMA issuer
+constexpr uint32_t kZTxBytes = C * NS * 2 + C * 4;
+// warps 0-3 epilogues, warp 4 TMA producer, warp 5 MMA issuer; with the output epilogue,
+// warps 6-7 write the output rows (TMEM lanes 64-127, as warps 2-3)
+__host__ __device__ constexpr int carry_threads(bool outg) { return outg ? 256 : 192; }
 
 // MN-major, unswizzled B operand with N = NS (32) columns: 8 x 8 core matrices of 128 bytes
 // (8 K-rows of 16 bytes); the NS / 8 core matrices of one group of 8 K-rows sit 128 bytes
@@ -686,7 +712,8 @@ __device__ __forceinline__ void store_op_row(f16* op, int k, const float* v, flo
 //   b: K_hat^T Delta~    (M=128, 4 MMAs)  -> D_b          state update
 //   c: [0; P] Delta      (M=128, 4 MMAs)  -> D_c[c % nb]  rows 64-127 P Delta
 // Epilogue threads 0-63 turn D_a rows into Delta, Delta~; all 128 update the state rows
-// from D_b; threads 64-127 write the output rows of chunk c while chunk c+1's MMAs run.
+// from D_b; without OUTG, threads 64-127 write the output rows of chunk c while chunk
+// c+1's MMAs run.
 // The two sides meet only through mbarriers (h0_ready, d_ready: one arrival per epilogue
 // warp, after its threads' shared-memory writes and proxy fences; the output warps
 // arrive on d_ready as soon as they have read the chunk's scalars, then
@@ -696,14 +723,16 @@ __device__ __forceinline__ void store_op_row(f16* op, int k, const float* v, flo
 // OUTG adds the output epilogue out = o rsqrt(mean(o^2) + eps) (1 + w) sigmoid(z) over the
 // 128 values of a head, which live in the head's four slice CTAs: those run as one
 // thread-block cluster (cluster rank = slice), and each output row's four partial sums of
-// squares cross over distributed shared memory, announced by remote mbarrier arrivals.
-// To keep that exchange off the serial chain the output warps write chunk c-2 (not c-1)
-// while chunk c's Delta and state MMA run, so D_a and D_c rotate over three buffers
-// (nb = 3) instead of two.
+// squares cross over distributed shared memory by bulk copies.  Two extra warps (6-7, on
+// TMEM lanes 64-127 like warps 2-3) do all of the output work, so that none of it sits
+// on the serial chain: the producer streams each chunk's z tile and row scalars into a
+// ring of NZ slots, D_a and D_c rotate over three buffers, and the MMA warp reuses a
+// buffer only after the output warps release it (ofree).
 template <bool OUTG>
-__global__ void __launch_bounds__(kCarryThreads, 1)
+__global__ void __launch_bounds__(carry_threads(OUTG), 1)
 chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qk,
                    const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_u,
+                   const __grid_constant__ CUtensorMap tm_z,
                    const float* __restrict__ SCg, const int32_t* __restrict__ cu,
                    const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HK, int HV,
                    const float* __restrict__ h0, float* __restrict__ hT, bf16* __restrict__ o,
@@ -745,13 +774,18 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         if (OUTG) {   // one local arrival per use, plus the peers' bulk copies as transactions
             tc::mbar_init(&S.obar[0], 1);
             tc::mbar_init(&S.obar[1], 1);
+            for (int i = 0; i < 3; ++i) tc::mbar_init(&S.ofree[i], 2);   // one per output warp
+            for (int i = 0; i < NZ; ++i) {
+                tc::mbar_init(&S.zfull[i], 1);
+                tc::mbar_init(&S.zempty[i], 2);
+            }
         }
         tc::fence_mbar_init();
         S.abort = 0;
     }
     if (OUTG && tid < NS) S.onw[tid] = 1.f + norm_w[vs * NS + tid];   // the (1 + w) factor
     // zero rows 0-63 of the P operands (the producer only ever writes rows 64-127)
-    for (int e = tid; e < NSTAGE * 64 * 64 / 8; e += kCarryThreads) {
+    for (int e = tid; e < NSTAGE * 64 * 64 / 8; e += carry_threads(OUTG)) {
         const int st = e / (64 * 64 / 8), r = e % (64 * 64 / 8);
         reinterpret_cast<uint4*>(S.st[st].P)[r] = make_uint4(0, 0, 0, 0);
     }
@@ -787,6 +821,17 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 tc::tma_load_2d(&B.P[64 * 64], &tm_p, &S.full[st], 0, row);
                 tc::tma_load_2d(B.U, &tm_u, &S.full[st], vs * NS, row);
                 tc::bulk_load(B.SC, SCg + ((size_t)cid * HV + h) * SC_FLOATS, SC_FLOATS * 4, &S.full[st]);
+                if (OUTG) {   // the chunk's z tile and per-row scalars, for the output warps
+                    const int k = c % NZ;
+                    if (c >= NZ && !tc::mbar_wait(&S.zempty[k], (uint32_t)(((c / NZ) - 1) & 1))) {
+                        record_timeout(status);
+                        S.abort = 1;
+                    }
+                    if (S.abort) break;
+                    tc::mbar_expect_tx(&S.zfull[k], kZTxBytes);
+                    tc::tma_load_3d(S.zr[k].z, &tm_z, &S.zfull[k], vs * NS, h, (int)(bos + (int64_t)C * c));
+                    tc::bulk_load(S.zr[k].a, SCg + ((size_t)cid * HV + h) * SC_FLOATS, C * 4, &S.zfull[k]);
+                }
             }
         }
     } else if (warp == 5) {
@@ -803,6 +848,11 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 ok = ok && tc::mbar_wait_spin(&S.h0_ready, c & 1);
                 if (!ok || S.abort) {
                     if (!ok) record_timeout(status);
+                    S.abort = 1;
+                    break;
+                }
+                if (OUTG && c >= nb && !tc::mbar_wait_spin(&S.ofree[c % nb], (uint32_t)(((c / nb) - 1) & 1))) {
+                    record_timeout(status);
                     S.abort = 1;
                     break;
                 }
@@ -837,7 +887,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 tc::mma_commit(&S.empty[st]);   // the stage's operands are consumed
             }
         }
-    } else {
+    } else if (warp < 4) {
         // ---------------- epilogues: 128 threads, thread t <-> TMEM lane t ------------------
         const int t = tid;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -857,84 +907,35 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         tc::named_bar(1, 128);
         const float inv_sc = pow2_above(fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3])));
         const float sc = 1.f / inv_sc;
+        if (OUTG) {   // publish the scale to the output warps
+            if (t == 0) S.inv_sc = inv_sc;
+            tc::named_bar_arrive(3, 128 + 64);
+        }
         store_op_row(S.H0[0], t, Hr, sc);
         tc::fence_async_smem();
+        tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&S.h0_ready);
+        if (lane == 0) tc::mbar_arrive(&S.h0_ready);   // phase 0: the initial state operand
+
         bool ok = true;
-        float a_prev = 0.f;          // per-row scalar, length and first token of the chunk whose
-        int cn_prev = 0;             //   output is written next (plain: the previous chunk;
-        int64_t tok_prev = 0;        //   OUTG: two chunks back, its successor in the *_nxt copies)
-        float a_nxt = 0.f;
-        int cn_nxt = 0;
-        int64_t tok_nxt = 0;
-        // OUTG: the gate inputs z of this row's values for the next chunk whose output is
-        // written, loaded one output call ahead so that their latency is off the chain
-        uint4 zpre[NS / 8];
-        auto load_z = [&](int64_t tok0, int rows) {
+        float a_prev = 0.f;          // plain: per-row scalar, length and first token of the
+        int cn_prev = 0;             //   previous chunk, whose output rows are written next
+        int64_t tok_prev = 0;
+        // plain: output rows of chunk cc (threads 64-127, row t - 64), from D_a and D_c
+        // buffer cc % nb, written under the next chunk's Delta epilogue and state MMA
+        auto write_output = [&](int cc) -> bool {
             const int i = t - 64;
-            if (OUTG && i < rows) {
-                const uint4* zr = reinterpret_cast<const uint4*>(zg + ((tok0 + i) * HV + h) * D + vs * NS);
-#pragma unroll
-                for (int qq = 0; qq < NS / 8; ++qq) zpre[qq] = zr[qq];
-            }
-        };
-        // output rows of chunk cc (threads 64-127, row t - 64), from D_a and D_c buffer cc % nb;
-        // OUTG with pre set then starts the z loads of the chunk held in the *_nxt copies
-        auto write_output = [&](int cc, bool pre) -> bool {
-            const int i = t - 64;
-            bool good = tc::mbar_wait(&S.bar_o[cc % nb], (uint32_t)((cc / nb) & 1));
+            const bool good = tc::mbar_wait(&S.bar_o[cc % nb], (uint32_t)((cc / nb) & 1));
             tc::tc_fence_after();
             const uint32_t par = (uint32_t)(cc % nb) * 32;
             float q[NS], z[NS];
             tc::tmem_ld32(tA + par + lane_base, q);
             tc::tmem_ld32(tC + par + lane_base, z);
             tc::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < NS; ++j) q[j] = fmaf(a_prev, q[j], z[j]) * inv_sc;   // the core output
-            if (OUTG) {
-                // this slice's sum of squares per row; the 64 rows go to each other slice CTA of
-                // the head in one bulk copy, which completes on that CTA's barrier
-                float ps = 0.f;
-#pragma unroll
-                for (int j = 0; j < NS; ++j) ps = fmaf(q[j], q[j], ps);
-                const int p = cc & 1;
-                S.oloc[p][i] = ps;
-                tc::fence_async_smem();
-                tc::named_bar(2, 64);   // the output warps' 64 rows are in oloc
-                if (t == 64) {
-                    tc::mbar_expect_tx(&S.obar[p], (nslices - 1) * C * 4);
-#pragma unroll
-                    for (int rk = 0; rk < nslices; ++rk)
-                        if (rk != vs)
-                            tc::bulk_copy_to_peer(tc::cluster_map(tc::smem_u32(&S.opart[p][vs][0]), rk), S.oloc[p], C * 4,
-                                                  tc::cluster_map(tc::smem_u32(&S.obar[p]), rk));
-                }
-                good = tc::mbar_wait_cluster(&S.obar[p], (uint32_t)((cc >> 1) & 1)) && good;
-                float ss = ps;
-#pragma unroll
-                for (int rk = 0; rk < nslices; ++rk)
-                    if (rk != vs) ss += S.opart[p][rk][i];
-                const float inv_rms = rsqrtf(ss * (1.f / D) + eps);
-                if (i < cn_prev) {
-#pragma unroll
-                    for (int qq = 0; qq < NS / 8; ++qq) {
-                        const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&zpre[qq]);
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const float2 zz = __bfloat1622float2(e[e2]);
-                            const int j = qq * 8 + e2 * 2;
-                            q[j] = q[j] * inv_rms * S.onw[j] * sigmoid_fast(zz.x);
-                            q[j + 1] = q[j + 1] * inv_rms * S.onw[j + 1] * sigmoid_fast(zz.y);
-                        }
-                    }
-                }
-                if (pre) load_z(tok_nxt, cn_nxt);
-            }
             if (i < cn_prev) {
                 __align__(16) bf16 ob[NS];
 #pragma unroll
-                for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(q[j]);
+                for (int j = 0; j < NS; ++j) ob[j] = __float2bfloat16_rn(fmaf(a_prev, q[j], z[j]) * inv_sc);
                 uint4* dst = reinterpret_cast<uint4*>(o + ((tok_prev + i) * HV + h) * D + vs * NS);
 #pragma unroll
                 for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
@@ -949,7 +950,6 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
             const int cn = (int)(rem < C ? rem : C);
             ok = tc::mbar_wait(&S.full[st], rr & 1);
             const float gC = B.SC[SC_GC];
-            float a_cur = 0.f;
             if (warp < 2) {
                 // ---- Delta rows (threads 0-63) ----------------------------------------------
                 ok = tc::mbar_wait(&S.bar_a, c & 1) && ok;
@@ -976,27 +976,16 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&S.d_ready);
             } else {
-                // ---- output warps: the chunk's scalars, then the output rows of an earlier
-                //      chunk under this chunk's Delta epilogue and state MMA: plain, chunk
-                //      c - 1; OUTG, chunk c - 2, so that its cluster exchange has a whole chunk
-                //      of slack (D_a, D_c of chunk c - 2 live until chunk c + 1's MMAs) ----------
-                a_cur = B.SC[t - 64];
+                // ---- warps 2-3: the chunk's scalars; plain, then the previous chunk's output
+                //      rows under this chunk's Delta epilogue and state MMA --------------------
+                const float a_cur = OUTG ? 0.f : B.SC[t - 64];
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&S.d_ready);   // the stage's scalars are read
                 if (!OUTG) {
-                    if (c > 0) ok = write_output(c - 1, false) && ok;
+                    if (c > 0) ok = write_output(c - 1) && ok;
                     a_prev = a_cur;
                     cn_prev = cn;
                     tok_prev = tok;
-                } else {
-                    if (c > 1) ok = write_output(c - 2, true) && ok;
-                    else if (c == 1) load_z(tok_nxt, cn_nxt);   // chunk 0's
-                    a_prev = a_nxt;
-                    cn_prev = cn_nxt;
-                    tok_prev = tok_nxt;
-                    a_nxt = a_cur;
-                    cn_nxt = cn;
-                    tok_nxt = tok;
                 }
             }
             // ---- state rows (all 128) ---------------------------------------------------------
@@ -1016,22 +1005,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
             if (lane == 0) tc::mbar_arrive(&S.h0_ready);
             if (S.abort) ok = false;
         }
-        if (warp >= 2) {   // output rows of the chunks still pending
-            if (OUTG) {
-                if (ok && nch > 1) {
-                    ok = write_output(nch - 2, true);
-                    a_prev = a_nxt;
-                    cn_prev = cn_nxt;
-                    tok_prev = tok_nxt;
-                } else if (nch == 1) {
-                    load_z(tok_nxt, cn_nxt);
-                    a_prev = a_nxt;
-                    cn_prev = cn_nxt;
-                    tok_prev = tok_nxt;
-                }
-            }
-            if (ok && nch > 0) ok = write_output(nch - 1, false);
-        }
+        if (!OUTG && warp >= 2 && ok && nch > 0) ok = write_output(nch - 1);   // the last chunk's rows
         if (!ok) {
             record_timeout(status);
             S.abort = 1;
@@ -1039,12 +1013,94 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
 #pragma unroll
             for (int j = 0; j < NS; ++j) hT[hrow + j] = Hr[j];
         }
+    } else if (OUTG) {
+        // ---------------- output warps 6-7: row i = TMEM lane 64 + i of D_a and D_c ----------
+        // out = o rsqrt(mean(o^2) + eps) (1 + w) sigmoid(z) per row over the head's 128
+        // values: this slice's sum of squares goes to the other three slice CTAs of the
+        // cluster in one bulk copy per peer, completing on their barrier obar[chunk parity]
+        const int i = tid - 192;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        tc::named_bar(3, 128 + 64);   // the state warps have published the data scale
+        const float inv_sc = S.inv_sc;
+        float wn[NS];   // 1 + w
+#pragma unroll
+        for (int j = 0; j < NS; ++j) wn[j] = S.onw[j];
+        for (int cc = 0; cc < nch; ++cc) {
+            const int k = cc % NZ, p = cc & 1;
+            const int64_t tok = bos + (int64_t)C * cc;
+            const int64_t rem = len - (int64_t)C * cc;
+            const int cn = (int)(rem < C ? rem : C);
+            bool good = tc::mbar_wait(&S.zfull[k], (uint32_t)((cc / NZ) & 1));
+            good = tc::mbar_wait(&S.bar_o[cc % nb], (uint32_t)((cc / nb) & 1)) && good;
+            tc::tc_fence_after();
+            const uint32_t par = (uint32_t)(cc % nb) * 32;
+            float q[NS], zc[NS];
+            tc::tmem_ld32(tA + par + lane_base, q);
+            tc::tmem_ld32(tC + par + lane_base, zc);
+            tc::tmem_wait_ld();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&S.ofree[cc % nb]);   // the buffer may take chunk cc + nb
+            const float a = S.zr[k].a[i];
+            float ps = 0.f;
+#pragma unroll
+            for (int j = 0; j < NS; ++j) {   // the core output, then its sum of squares
+                q[j] = fmaf(a, q[j], zc[j]) * inv_sc;
+                ps = fmaf(q[j], q[j], ps);
+            }
+            S.oloc[p][i] = ps;
+            tc::fence_async_smem();
+            tc::named_bar(2, 64);   // the 64 rows are in oloc
+            if (i == 0) {
+                tc::mbar_expect_tx(&S.obar[p], (nslices - 1) * C * 4);
+#pragma unroll
+                for (int rk = 0; rk < nslices; ++rk)
+                    if (rk != vs)
+                        tc::bulk_copy_to_peer(tc::cluster_map(tc::smem_u32(&S.opart[p][vs][0]), rk), S.oloc[p], C * 4,
+                                              tc::cluster_map(tc::smem_u32(&S.obar[p]), rk));
+            }
+            good = tc::mbar_wait_cluster(&S.obar[p], (uint32_t)((cc >> 1) & 1)) && good;
+            float ss = ps;
+#pragma unroll
+            for (int rk = 0; rk < nslices; ++rk)
+                if (rk != vs) ss += S.opart[p][rk][i];
+            const float inv_rms = rsqrtf(ss * (1.f / D) + eps);
+            if (i < cn) {
+                const uint4* zrow = reinterpret_cast<const uint4*>(S.zr[k].z + i * NS);
+                __align__(16) bf16 ob[NS];
+#pragma unroll
+                for (int qq = 0; qq < NS / 8; ++qq) {
+                    const uint4 u = zrow[qq];
+                    const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const float2 zz = __bfloat1622float2(e[e2]);
+                        const int j = qq * 8 + e2 * 2;
+                        ob[j] = __float2bfloat16_rn(q[j] * inv_rms * wn[j] * sigmoid_fast(zz.x));
+                        ob[j + 1] = __float2bfloat16_rn(q[j + 1] * inv_rms * wn[j + 1] * sigmoid_fast(zz.y));
+                    }
+                }
+                uint4* dst = reinterpret_cast<uint4*>(o + ((tok + i) * HV + h) * D + vs * NS);
+#pragma unroll
+                for (int qq = 0; qq < NS / 8; ++qq) dst[qq] = reinterpret_cast<const uint4*>(ob)[qq];
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&S.zempty[k]);   // the slot may take chunk cc + NZ
+            // both output warps leave together: a failed wait or an abort elsewhere
+            if (tc::named_bar_any(2, 64, !good || S.abort)) {
+                if (i == 0) record_timeout(status);
+                S.abort = 1;
+                break;
+            }
+        }
     }
     tc::tc_fence_before();
     __syncthreads();
     if (S.abort && tid == 0) {
         // let copies already issued land before the shared memory is released
         for (int i = 0; i < NSTAGE; ++i) (void)tc::mbar_wait(&S.full[i], 0, 50000000ull);
+        if (OUTG)
+            for (int i = 0; i < NZ; ++i) (void)tc::mbar_wait(&S.zfull[i], 0, 50000000ull);
     }
     __syncthreads();
     if (OUTG) tc::cluster_sync();   // no CTA leaves while a peer may still write its shared memory
@@ -1212,16 +1268,23 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
         e = cudaFuncSetAttribute(chunk_carry_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kCarrySmemBytes);
         if (e != cudaSuccess) return e;
-        chunk_carry_kernel<false><<<blocks, kCarryThreads, kCarrySmemBytes, s>>>(
-            tw, tqk, tp, tu, SC, a.cu, chunk_off, a.T, a.n_seqs, a.HK, a.HV, a.h0, a.hT, (bf16*)a.o, nullptr,
+        chunk_carry_kernel<false><<<blocks, carry_threads(false), kCarrySmemBytes, s>>>(
+            tw, tqk, tp, tu, tw, SC, a.cu, chunk_off, a.T, a.n_seqs, a.HK, a.HV, a.h0, a.hT, (bf16*)a.o, nullptr,
             nullptr, 0.f, a.status);
     } else {   // the head's four column slices as one cluster (output epilogue)
+        // z [tokens, HV, Dv] bf16: one slice's 32 values of one head for 64 tokens per tile
+        CUtensorMap tz;
+        cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.HV, tok};
+        cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.HV * D * 2};
+        cuuint32_t box[3] = {NS, 1, 64};
+        if (!make_map(&tz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.z, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
         e = cudaFuncSetAttribute(chunk_carry_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kCarrySmemBytes);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(blocks);
-        cfg.blockDim = dim3(kCarryThreads);
+        cfg.blockDim = dim3(carry_threads(true));
         cfg.dynamicSmemBytes = kCarrySmemBytes;
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
@@ -1231,7 +1294,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, chunk_carry_kernel<true>, tw, tqk, tp, tu, (const float*)SC, a.cu,
+        e = cudaLaunchKernelEx(&cfg, chunk_carry_kernel<true>, tw, tqk, tp, tu, tz, (const float*)SC, a.cu,
                                (const int32_t*)chunk_off, a.T, a.n_seqs, a.HK, a.HV, a.h0, a.hT, (bf16*)a.o,
                                (const bf16*)a.z, a.norm_w, a.eps, a.status);
         if (e != cudaSuccess) return e;

@@ -112,21 +112,25 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const vo
     asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(dst_cluster), "r"(smem_u32(src)), "r"(bytes), "r"(mbar_cluster) : "memory");
 }
-// Bounded wait (acquire, cluster scope) on this CTA's mbarrier that other CTAs arrive on.
+// Bounded wait (acquire, cluster scope) on this CTA's mbarrier that other CTAs arrive on or
+// complete transactions on.  The clock is read once per 32 polls: reading it on every poll
+// measurably slows the other warps of the SM.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
                                                   uint64_t timeout_ns = 2000000000ull) {
     const uint32_t addr = smem_u32(bar);
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(addr), "r"(parity)
-            : "memory");
-        if (done) return true;
+        for (int i = 0; i < 32; ++i) {
+            uint32_t done;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(done)
+                : "r"(addr), "r"(parity)
+                : "memory");
+            if (done) return true;
+        }
         if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
 }
@@ -143,6 +147,11 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Arrive on a named barrier without waiting (the waiting side uses named_bar with the same
+// total thread count); orders this thread's earlier memory accesses before the waiters' later ones.
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---- TMA ------------------------------------------------------------------------------
