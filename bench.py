@@ -404,6 +404,32 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     barrier()
     gated_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
     del zd, wd
+
+    # ---------------- the convolution prologue: raw q | k | v projections -> q, k, v ----------------
+    C = 2 * HK * D + HV * D
+    xr, cw, cst = I.conv_prefill_inputs(T, 1, HK, HV, D, I.BF16, replica_seed(88, rank), True)
+    xd, cwd = dev_t(xr).view(1, T, C), dev_t(cw)
+    csd = dev_t(np.ascontiguousarray(cst.transpose(0, 2, 1)))
+    cq, ck, cv, cso = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(csd)
+    del xr
+
+    def conv_step():
+        G.gdn_conv_prefill(xd, cwd, HK, HV, D, D, conv_state_in=csd, conv_act=1, q=cq, k=ck, v=cv,
+                           conv_state_out=cso)
+
+    for _ in range(3):
+        conv_step()
+    barrier()
+    c0 = torch.cuda.Event(enable_timing=True)
+    c1 = torch.cuda.Event(enable_timing=True)
+    c0.record()
+    for _ in range(args.steps):
+        conv_step()
+    c1.record()
+    barrier()
+    conv_ms = max_over_ranks(c0.elapsed_time(c1) / args.steps)
+    conv_bytes = 2 * T * C * 2 + C * 16 + 2 * 3 * C * 4   # x in, q | k | v out, weights, states
+    del xd, cwd, csd, cq, ck, cv, cso
     flops = prefill_flops_per_token(HK, HV, D, BT) * T
     pbytes = prefill_bytes_per_token(HK, HV, D) * T + HV * D * D * 4
     tflops = flops / (kernel_ms * 1e-3) / 1e12
@@ -429,6 +455,12 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
                                  "epilogue (eps 1e-6) fused into the state carry; gates precomputed",
                          "ms_per_call": gated_ms, "tokens_per_s": whole_job_rate(world, T, gated_ms),
                          "core_prefill_ms_per_call": kernel_ms},
+        "conv_prologue": {"what": "gdn_conv_prefill: kernel-4 causal convolution (SiLU) from the raw q|k|v "
+                                  "projections [T, 8192] bf16 to the prefill's q, k, v, state carried in and out",
+                          "ms_per_call": conv_ms, "bytes_per_call": conv_bytes,
+                          "achieved_gbs": conv_bytes / (conv_ms * 1e-3) / 1e9,
+                          "frac": conv_bytes / (conv_ms * 1e-3) / 1e9 / P["hbm_gbs"],
+                          "peak_kind": f"{pk} copy bandwidth"},
     }
 
 

@@ -52,6 +52,7 @@ _SIGS = {
     "gdn_decode_step": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                          _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_conv_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
     "gdn_decode_step_fused": ([_vp, ctypes.c_int, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_int, _vp, _vp, _vp,
                                _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_chunk_prefill_host_workspace_bytes": ([_i32, _i64, _i32, _i32, _i32, _i32, _i32, ctypes.c_int,
@@ -59,6 +60,8 @@ _SIGS = {
     "gdn_chunk_prefill_host": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i64,
                                 _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i64, _vp, _vp, _vp, _sz, _vp],
                                ctypes.c_int),
+    "gdn_conv_prefill": ([_vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32,
+                          _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "gdn_decode_step_gated": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32,
                                _i32, _i32, _i32, _f32, _i32, _vp, _vp], ctypes.c_int),
 }
@@ -330,6 +333,48 @@ def gdn_decode_step_fused(x, conv_w, conv_state_in, a, b, A_log, dt_bias, state,
                                      int(bool(qk_l2norm)), _ptr(o), _stream())
     _check(st, "gdn_decode_step_fused")
     return o, conv_state_out
+
+
+def gdn_conv_prefill(x, conv_w, HK: int, HV: int, Dk: int = 128, Dv: int = 128, conv_state_in=None,
+                     cu_seqlens=None, conv_act: int = 1, output_conv_state: bool = True,
+                     q=None, k=None, v=None, conv_state_out=None):
+    """The prefill prologue: x [B, T, C] raw q | k | v projections (C = 2 HK Dk + HV Dv;
+    packed: B = 1 with cu_seqlens int32 [N + 1]); conv_w [C, 4]; conv_state_in [N, 3, C]
+    fp32 or None.  Returns (q [B, T, HK, Dk], k, v [B, T, HV, Dv], conv_state_out [N, 3, C]
+    or None)."""
+    B, T, C = x.shape
+    if C != 2 * HK * Dk + HV * Dv or conv_w.shape != (C, 4) or conv_w.dtype != torch.float32:
+        raise ValueError("x must be [B, T, 2 HK Dk + HV Dv] and conv_w fp32 [C, 4]")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if conv_state_in is not None and (conv_state_in.shape != (N, 3, C) or conv_state_in.dtype != torch.float32):
+        raise ValueError("conv_state_in must be fp32 [N, 3, C]")
+    if q is None:
+        q = torch.empty((B, T, HK, Dk), dtype=x.dtype, device=x.device)
+    if k is None:
+        k = torch.empty((B, T, HK, Dk), dtype=x.dtype, device=x.device)
+    if v is None:
+        v = torch.empty((B, T, HV, Dv), dtype=x.dtype, device=x.device)
+    if conv_state_out is None and output_conv_state:
+        conv_state_out = torch.empty((N, 3, C), dtype=torch.float32, device=x.device)
+    st = lib().gdn_conv_prefill(_ptr(x), _dtype_code(x), _ptr(conv_w), _ptr(conv_state_in), _ptr(cu_seqlens),
+                                B, T, N, HK, HV, Dk, Dv, int(conv_act), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(conv_state_out), _stream())
+    _check(st, "gdn_conv_prefill")
+    return q, k, v, conv_state_out
+
+
+def gdn_conv_status() -> int:
+    """Synchronise the device, return the convolution kernel's error word and clear it."""
+    word = _i32(0)
+    st = lib().gdn_conv_status(ctypes.byref(word))
+    if st not in (0, 8):
+        _check(st, "gdn_conv_status")
+    return int(word.value)
 
 
 def gdn_decode_status() -> int:

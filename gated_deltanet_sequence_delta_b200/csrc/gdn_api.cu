@@ -291,6 +291,51 @@ gdn_status gdn_decode_step_fused(const void* x, gdn_dtype io_dtype, const float*
                                                qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
 }
 
+gdn_status gdn_conv_prefill(const void* x, gdn_dtype io_dtype, const float* conv_w, const float* conv_state_in,
+                            const int32_t* cu_seqlens, int32_t B, int64_t T, int32_t n_seqs, int32_t HK,
+                            int32_t HV, int32_t Dk, int32_t Dv, int32_t conv_act, void* q, void* k, void* v,
+                            float* conv_state_out, void* stream) {
+    if (B < 0 || T < 0 || n_seqs < 0 || HK <= 0 || HV <= 0) return GDN_ERR_SHAPE;
+    if (cu_seqlens ? B != 1 : n_seqs != B) return GDN_ERR_SHAPE;
+    if (!dtype_ok(io_dtype) || !head_dim_ok(Dk) || !head_dim_ok(Dv) || (conv_act != 0 && conv_act != 1))
+        return GDN_ERR_UNSUPPORTED;
+    const int64_t n_tok = (int64_t)B * T;
+    const size_t C = (size_t)2 * HK * Dk + (size_t)HV * Dv;
+    if (C > (size_t)INT32_MAX || (n_tok > 0 && (size_t)n_tok > SIZE_MAX / (C * 4))) return GDN_ERR_SHAPE;
+    if (n_seqs == 0) return GDN_OK;
+    if (!conv_w || (n_tok > 0 && (!x || !q || !k || !v))) return GDN_ERR_NULL;
+    const void* ptrs[] = {x, conv_w, conv_state_in, cu_seqlens, q, k, v, conv_state_out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t es = esize(io_dtype), qk = (size_t)HK * Dk;
+    const Range rx{x, (size_t)n_tok * C * es}, rw{conv_w, C * 16};
+    const Range rci{conv_state_in, conv_state_in ? (size_t)n_seqs * C * 12 : 0};
+    const Range rcu{cu_seqlens, cu_seqlens ? (size_t)(n_seqs + 1) * 4 : 0};
+    const Range rq{q, (size_t)n_tok * qk * es}, rk{k, (size_t)n_tok * qk * es};
+    const Range rv{v, (size_t)n_tok * HV * Dv * es};
+    const Range rco{conv_state_out, conv_state_out ? (size_t)n_seqs * C * 12 : 0};
+    for (Range out : {rq, rk, rv, rco})
+        for (Range in : {rx, rw, rci, rcu})
+            if (overlap(out, in)) return GDN_ERR_ALIAS;
+    if (overlap(rq, rk) || overlap(rq, rv) || overlap(rk, rv) || overlap(rq, rco) || overlap(rk, rco) ||
+        overlap(rv, rco))
+        return GDN_ERR_ALIAS;
+    return cuda_status(gdn::launch_conv_prefill(x, io_dtype == GDN_BF16, conv_w, conv_state_in, cu_seqlens, n_tok,
+                                                T, n_seqs, (int)C, (int)qk, conv_act, q, k, v, conv_state_out,
+                                                (cudaStream_t)stream));
+}
+
+gdn_status gdn_conv_status(int32_t* device_error) {
+    if (!device_error) return GDN_ERR_NULL;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e);
+    int32_t word = 0;
+    e = gdn::read_conv_error(&word, true);
+    if (e != cudaSuccess) return cuda_status(e);
+    *device_error = word;
+    return word ? GDN_ERR_DEVICE : GDN_OK;
+}
+
 gdn_status gdn_decode_status(int32_t* device_error) {
     if (!device_error) return GDN_ERR_NULL;
     cudaError_t e = cudaDeviceSynchronize();

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -96,6 +97,21 @@ struct DecodeConv {
 // Dk = Dv = 128 only.
 cudaError_t launch_decode_conv(bool bf16, const DecodeConv& conv, const DecodeGates& gates, float* state, int B,
                                int HK, int HV, float scale, int l2norm, void* o, cudaStream_t s);
+
+// Tiled tensor map (element strides 1, no interleave, zero fill out of range); false if the
+// driver entry point is missing or the encoder rejects the arguments.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw);
+
+// Causal depthwise convolution of kernel 4 over whole sequences (dense when cu is null:
+// n_seqs sequences of T tokens): x [n_tokens, C] with C = 2 qk + (v channels), written to
+// q, k [n_tokens, qk] and v [n_tokens, C - 2 qk]; states [n_seqs, 3, C] fp32 tap-major.
+cudaError_t launch_conv_prefill(const void* x, bool bf16, const float* w, const float* state_in,
+                                const int32_t* cu, int64_t n_tokens, int64_t T, int n_seqs, int C, int qk,
+                                int act, void* q, void* k, void* v, float* state_out, cudaStream_t s);
+
+// Read (and on request clear) the device word the bf16 convolution kernel sets on a timeout.
+cudaError_t read_conv_error(int32_t* out, bool reset);
 
 // Read (and on request clear) the device word a staged decode launch sets on a timeout.
 cudaError_t read_decode_error(int32_t* out, bool reset);

@@ -197,6 +197,19 @@ def outgate_inputs(n_tokens: int, HV: int, Dv: int, io_dtype: str, seed: int):
     return z, w
 
 
+def conv_prefill_inputs(n_tokens: int, n_seqs: int, HK: int, HV: int, D: int, io_dtype: str, seed: int,
+                        with_state: bool = True):
+    """Raw q | k | v projection rows x [n_tokens, C] (C = 2 HK D + HV D) ~ N(0, 1) in the io
+    dtype, convolution weights conv_w [C, 4] ~ N(0, 0.5^2) fp32 and initial convolution
+    states [n_seqs, C, 3] ~ N(0, 1) fp32 (None without ``with_state``): the recipe of the
+    decode step from raw projections, over whole sequences."""
+    C = 2 * HK * D + HV * D
+    x = _normal_rows(_rng(seed, 400, 1), n_tokens, (C,), io_dtype, False)
+    conv_w = (0.5 * _rng(seed, 400, 2).standard_normal((C, 4), dtype=np.float32)).astype(np.float32)
+    state = _rng(seed, 400, 3).standard_normal((n_seqs, C, 3), dtype=np.float32) if with_state else None
+    return x, conv_w, state
+
+
 def varlen_lengths(seed: int, total: int = 65536, lo: int = 512, hi: int = 8192) -> np.ndarray:
     """Sequence lengths ~ U_int[lo, hi] until they sum to ``total`` (last one truncated)."""
     rng = _rng(seed, _STREAM["lens"])

@@ -177,6 +177,50 @@ GDN_API gdn_status gdn_chunk_prefill_outgate(const void* q, const void* k, const
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * gdn_conv_prefill -- the prefill prologue: the causal depthwise convolution of kernel 4
+ * that the "Gated DeltaNet ... Qwen3-next" page (section 3.1) places before the gated
+ * update (kernel size from the tutorial page, section 6, linear_conv_kernel_dim = 4),
+ * over whole sequences, from the raw q | k | v projections to the q, k, v inputs of
+ * gdn_chunk_prefill, with the rolling state of each sequence carried in and out:
+ *   y_t = w0 x_{t-3} + w1 x_{t-2} + w2 x_{t-1} + w3 x_t per channel, then identity or SiLU.
+ * Sequences as gdn_chunk_prefill: dense (cu_seqlens == NULL, B sequences of T tokens,
+ * n_seqs == B) or packed (B == 1, T total tokens, n_seqs sequences in cu_seqlens).
+ *   x      [B, T, C] io_dtype, C = 2 HK Dk + HV Dv: q channels (head-major), then k, then v
+ *                                                                              (read)
+ *   conv_w [C, 4] fp32, taps oldest first                                      (read)
+ *   conv_state_in  [n_seqs, 3, C] fp32, the three inputs before each sequence, oldest
+ *          first, or NULL for zeros                                            (read)
+ *   conv_act  0: y;  1: SiLU, y / (1 + exp(-y))   (the pages name no activation)
+ *   q, k   [B, T, HK, Dk] io_dtype;  v [B, T, HV, Dv] io_dtype: y rounded to io_dtype
+ *                                                                              (written)
+ *   conv_state_out [n_seqs, 3, C] fp32, each sequence's three newest inputs (with the
+ *          carried state for sequences shorter than 3; a zero-length sequence passes its
+ *          state through), or NULL (written).  It is the conv_state_in of the next
+ *          prefill piece or of gdn_decode_step_fused.
+ * No output may overlap an input or another output (conv_state_out may not be
+ * conv_state_in).  cu_seqlens is not checked here (gdn_chunk_prefill checks the same
+ * table on the device); with a bad table the outputs are undefined, but every access
+ * stays inside the buffers the sizes describe.
+ * For bf16 the convolution runs as a persistent kernel fed by tile copies, whose waits are
+ * bounded; if one expires (no such case is known) the launch stops early and records
+ * GDN_DEVERR_TIMEOUT, which gdn_conv_status reports.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (Dk, Dv not 64 or 128), ALIAS, CUDA.
+ */
+GDN_API gdn_status gdn_conv_prefill(const void* x, gdn_dtype io_dtype, const float* conv_w,
+                                    const float* conv_state_in, const int32_t* cu_seqlens,
+                                    int32_t B, int64_t T, int32_t n_seqs,
+                                    int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t conv_act,
+                                    void* q, void* k, void* v, float* conv_state_out, void* stream);
+
+/*
+ * Synchronises the device, then reads and clears the device word of the convolution kernel
+ * (GDN_DEVERR_NONE or GDN_DEVERR_TIMEOUT, shared by every gdn_conv_prefill launch on that
+ * device) into *device_error.  Returns GDN_ERR_DEVICE if it is nonzero.
+ * Errors: NULL, CUDA.
+ */
+GDN_API gdn_status gdn_conv_status(int32_t* device_error);
+
+/*
  * Synchronises `stream`, then reads the device status word of a prefill
  * workspace into *device_error (GDN_DEVERR_*).  Returns GDN_ERR_DEVICE if it
  * is nonzero, GDN_ERR_CUDA if the synchronisation failed, else GDN_OK.

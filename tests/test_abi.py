@@ -203,8 +203,33 @@ def test_decode_fused_validation(L):
     assert call(a12=0) == 0                     # B = 0: nothing to do
 
 
+def test_conv_prefill_validation(L):
+    f = L.gdn_conv_prefill
+    # x, io, w, cs_in, cu, B, T, N, HK, HV, Dk, Dv, act, q, k, v, cs_out, stream
+    base = [A, 1, A + MB, A + 2 * MB, None, 2, 100, 2, 2, 4, 128, 128, 1, A + 8 * MB, A + 9 * MB, A + 10 * MB,
+            A + 11 * MB, None]
+    def call(**kw):
+        a = list(base)
+        for i, val in kw.items():
+            a[int(i[1:])] = val
+        return f(*a)
+    assert call(a0=None) == 1                   # x
+    assert call(a2=None) == 1                   # weights
+    assert call(a12=2) == 4                     # activation code
+    assert call(a10=96) == 4                    # head dim
+    assert call(a4=A + 12 * MB) == 2            # packed needs B = 1
+    assert call(a7=3) == 2                      # dense: n_seqs = B
+    assert call(a8=0) == 2                      # HK
+    assert call(a13=A + 8 * MB + 4) == 3        # q misaligned
+    assert call(a13=A) == 5                     # q over x
+    assert call(a16=A + 2 * MB) == 5            # conv_state_out over conv_state_in
+    assert call(a14=A + 8 * MB + 64) == 5       # k over q
+    assert call(a5=0, a7=0) == 0                # no sequences: nothing to do
+
+
 def test_decode_status_null(L):
     assert L.gdn_decode_status(None) == 1
+    assert L.gdn_conv_status(None) == 1
 
 
 def test_missing_library_fails_loudly(tmp_path):
