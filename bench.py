@@ -460,6 +460,7 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
                           "ms_per_call": conv_ms, "bytes_per_call": conv_bytes,
                           "achieved_gbs": conv_bytes / (conv_ms * 1e-3) / 1e9,
                           "frac": conv_bytes / (conv_ms * 1e-3) / 1e9 / P["hbm_gbs"],
+                          "traffic": _traffic().get("conv_prefill_bytes_per_launch"),
                           "peak_kind": f"{pk} copy bandwidth"},
     }
 
