@@ -284,6 +284,7 @@ struct PrepSmem {
     float M[64][65];
     float X[3][16][17];
     float rk[64], rq[64], G[64], bt[64], bgr[64], red[8];
+    float eu[64];   // rk_j exp(G_r - G_j), the token factor of the separated decays
     float ga[2][64], ba[2][64];   // prefetched g, beta of the (up to two) value heads
     uint64_t bar_load, bar_v, bar_mma;
     uint32_t tmem_base;
@@ -459,6 +460,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncthreads();
             if (tid < 64) S.bgr[tid] = S.bt[tid] * expf(S.G[tid]);
             const float Gl = S.G[63];   // padding adds 0, so this is G at the last token
+            // exp(G_i - G_j) = exp(G_i - G_r) exp(G_r - G_j) with G_r = G_last / 2: both
+            // factors stay inside fp32 range while G_last >= -160, and the row loops below
+            // then need no exponential per pair; deeper decays take exp(G_i - G_j) directly
+            const bool sep = Gl >= -160.f;
+            const float Gr = 0.5f * Gl;
+            if (sep) {
+                if (tid < 64) S.eu[tid] = S.rk[tid] * __expf(Gr - S.G[tid]);
+                __syncthreads();
+            }
             // ---- L (strictly lower) into M, P (lower incl. diagonal) out, scalars; the
             //      Gram row of this thread is read back from TMEM --------------------------
             {
@@ -469,11 +479,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (tid < 64) {
                     const int i = tid;
                     const float Gi = S.G[i], bi = S.bt[i] * rki;
+                    if (sep) {
+                        const float ai = i < cn ? bi * __expf(Gi - Gr) : 0.f;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        float v = 0.f;
-                        if (j < i && i < cn) v = bi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
-                        S.M[i][j] = v;
+                        for (int j = 0; j < 64; ++j) S.M[i][j] = j < i ? ai * S.eu[j] * row[j] : 0.f;
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) {
+                            float v = 0.f;
+                            if (j < i && i < cn) v = bi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
+                            S.M[i][j] = v;
+                        }
                     }
                     SCg[ch * SC_FLOATS + 64 + i] = i < cn ? expf(Gl - Gi) : 0.f;
                 } else {
@@ -482,6 +498,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     SCg[ch * SC_FLOATS + i] = i < cn ? scale * expf(Gi) : 0.f;
                     if (i == 0) SCg[ch * SC_FLOATS + SC_GC] = expf(Gl);
                     uint4* prow = reinterpret_cast<uint4*>(Pg + (ch * 64 + i) * 64);
+                    const float ai = sep && i < cn ? qi * __expf(Gi - Gr) : 0.f;
 #pragma unroll
                     for (int c8 = 0; c8 < 8; ++c8) {
                         __align__(16) f16 e[8];
@@ -489,7 +506,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         for (int t = 0; t < 8; ++t) {
                             const int j = c8 * 8 + t;
                             float v = 0.f;
-                            if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
+                            if (sep) v = j <= i ? ai * S.eu[j] * row[j] : 0.f;
+                            else if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
                             e[t] = __float2half_rn(v);
                         }
                         prow[c8] = *reinterpret_cast<const uint4*>(e);
