@@ -53,6 +53,8 @@ _SIGS = {
                          _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
     "gdn_conv_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_cp_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _i32, _i32, ctypes.c_int, _vp, _vp, _vp, _vp,
+                        _vp], ctypes.c_int),
     "gdn_decode_step_fused": ([_vp, ctypes.c_int, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_int, _vp, _vp, _vp,
                                _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_chunk_prefill_host_workspace_bytes": ([_i32, _i64, _i32, _i32, _i32, _i32, _i32, ctypes.c_int,
@@ -366,6 +368,28 @@ def gdn_conv_prefill(x, conv_w, HK: int, HV: int, Dk: int = 128, Dv: int = 128, 
                                 _ptr(conv_state_out), _stream())
     _check(st, "gdn_conv_prefill")
     return q, k, v, conv_state_out
+
+
+def gdn_cp_combine(A_all, B_all, o, c, rank: int, initial_state=None, start_state=None, final_state=None,
+                   output_final_state: bool = True):
+    """The exchange step of a context-parallel prefill: A_all, B_all [R, N, HV, 128, 128]
+    fp32 (every segment's transition and zero-start final state), o [N, T_seg, HV, 128]
+    (this segment's zero-start output, corrected in place) and c (its transition outputs).
+    Returns (start_state, final_state or None)."""
+    R, N, HV, Dk, Dv = A_all.shape
+    if B_all.shape != A_all.shape or A_all.dtype != torch.float32 or B_all.dtype != torch.float32:
+        raise ValueError("A_all, B_all must be fp32 [R, N, HV, Dk, Dv] of one shape")
+    T_seg = o.shape[1]
+    if o.shape != (N, T_seg, HV, Dv) or c.shape != o.shape or c.dtype != o.dtype:
+        raise ValueError("o, c must be [N, T_seg, HV, Dv] of one dtype")
+    if start_state is None:
+        start_state = torch.empty((N, HV, Dk, Dv), dtype=torch.float32, device=o.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, HV, Dk, Dv), dtype=torch.float32, device=o.device)
+    st = lib().gdn_cp_combine(_ptr(A_all), _ptr(B_all), _ptr(initial_state), R, int(rank), N, T_seg, HV, Dk, Dv,
+                              _dtype_code(o), _ptr(o), _ptr(c), _ptr(start_state), _ptr(final_state), _stream())
+    _check(st, "gdn_cp_combine")
+    return start_state, final_state
 
 
 def gdn_conv_status() -> int:

@@ -325,6 +325,31 @@ gdn_status gdn_conv_prefill(const void* x, gdn_dtype io_dtype, const float* conv
                                                 (cudaStream_t)stream));
 }
 
+gdn_status gdn_cp_combine(const float* A_all, const float* B_all, const float* initial_state, int32_t R,
+                          int32_t rank, int32_t n_seqs, int64_t T_seg, int32_t HV, int32_t Dk, int32_t Dv,
+                          gdn_dtype io_dtype, void* o, const void* c, float* start_state, float* final_state,
+                          void* stream) {
+    if (R < 1 || rank < 0 || rank >= R || n_seqs < 0 || T_seg < 0 || HV <= 0) return GDN_ERR_SHAPE;
+    if (!dtype_ok(io_dtype) || Dk != 128 || Dv != 128) return GDN_ERR_UNSUPPORTED;
+    if (n_seqs == 0) return GDN_OK;
+    if (!A_all || !B_all || !start_state || (T_seg > 0 && (!o || !c))) return GDN_ERR_NULL;
+    const void* ptrs[] = {A_all, B_all, initial_state, o, c, start_state, final_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t nh = (size_t)n_seqs * HV, mat = (size_t)Dk * Dv * 4, es = esize(io_dtype);
+    const Range rA{A_all, (size_t)R * nh * mat}, rB{B_all, (size_t)R * nh * mat};
+    const Range rh{initial_state, initial_state ? nh * mat : 0};
+    const Range ro{o, (size_t)T_seg * nh * Dv * es}, rc{c, (size_t)T_seg * nh * Dk * es};
+    const Range rs{start_state, nh * mat}, rf{final_state, final_state ? nh * mat : 0};
+    for (Range out : {ro, rs, rf})
+        for (Range in : {rA, rB, rh, rc})
+            if (overlap(out, in)) return GDN_ERR_ALIAS;
+    if (overlap(ro, rs) || overlap(ro, rf) || overlap(rs, rf)) return GDN_ERR_ALIAS;
+    return cuda_status(gdn::launch_cp_combine(A_all, B_all, initial_state, R, rank, n_seqs, T_seg, HV,
+                                              io_dtype == GDN_BF16, o, c, start_state, final_state,
+                                              (cudaStream_t)stream));
+}
+
 gdn_status gdn_conv_status(int32_t* device_error) {
     if (!device_error) return GDN_ERR_NULL;
     cudaError_t e = cudaDeviceSynchronize();

@@ -110,6 +110,14 @@ cudaError_t launch_conv_prefill(const void* x, bool bf16, const float* w, const 
                                 const int32_t* cu, int64_t n_tokens, int64_t T, int n_seqs, int C, int qk,
                                 int act, void* q, void* k, void* v, float* state_out, cudaStream_t s);
 
+// Context-parallel prefill, the exchange step: A_all, B_all [R, n_seqs, HV, 128, 128] (every
+// segment's transition and zero-start final state), h0 the sequence's initial states (may be
+// null); writes this rank's start states, the sequences' final states (may be null) and adds
+// H_start^T c_t to o in place (o, c [n_seqs, T_seg, HV, 128]).
+cudaError_t launch_cp_combine(const float* A_all, const float* B_all, const float* h0, int R, int rank, int n_seqs,
+                              int64_t T_seg, int HV, bool bf16, void* o, const void* c, float* start_state,
+                              float* final_state, cudaStream_t s);
+
 // Read (and on request clear) the device word the bf16 convolution kernel sets on a timeout.
 cudaError_t read_conv_error(int32_t* out, bool reset);
 

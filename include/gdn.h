@@ -221,6 +221,31 @@ GDN_API gdn_status gdn_conv_prefill(const void* x, gdn_dtype io_dtype, const flo
 GDN_API gdn_status gdn_conv_status(int32_t* device_error);
 
 /*
+ * gdn_cp_combine -- the exchange step of a context-parallel prefill, in which each of R
+ * ranks holds one consecutive segment of the same sequences (rank r the r-th segment of
+ * T_seg tokens).  Over a segment the rule is affine in the state it starts from (the
+ * product form of the update, "Gated DeltaNet" research log; H = S^T):
+ *     H_end = A H_start + B,   o_t = o0_t + H_start^T c_t,
+ * B and o0 being the segment's gdn_chunk_prefill from a zero state, A and c its
+ * gdn_chunk_prefill with v = 0 from H_start = I (A = the product of the segment's
+ * transitions, c_t = scale A_{<=t}^T q_t).  With every rank's (A, B) gathered, this call
+ * forms H_start(rank) by the scan H_start(0) = initial_state, H_start(r + 1) = A_r
+ * H_start(r) + B_r, the sequences' final states, and corrects o in place.
+ *   A_all, B_all  [R, n_seqs, HV, 128, 128] fp32, rank-major                     (read)
+ *   initial_state [n_seqs, HV, 128, 128] fp32, the state before segment 0, or NULL (read)
+ *   o             [n_seqs, T_seg, HV, 128] io_dtype: o0 in, the rank's outputs out
+ *   c             [n_seqs, T_seg, HV, 128] io_dtype                              (read)
+ *   start_state   [n_seqs, HV, 128, 128] fp32, H_start of this rank's segment   (written)
+ *   final_state   [n_seqs, HV, 128, 128] fp32, the state after segment R - 1, or NULL
+ * Dk = Dv = 128 only.  No output may overlap an input or another output.
+ * Errors: NULL, SHAPE (R, rank, sizes), ALIGN, UNSUPPORTED, ALIAS, CUDA.
+ */
+GDN_API gdn_status gdn_cp_combine(const float* A_all, const float* B_all, const float* initial_state,
+                                  int32_t R, int32_t rank, int32_t n_seqs, int64_t T_seg, int32_t HV,
+                                  int32_t Dk, int32_t Dv, gdn_dtype io_dtype, void* o, const void* c,
+                                  float* start_state, float* final_state, void* stream);
+
+/*
  * Synchronises `stream`, then reads the device status word of a prefill
  * workspace into *device_error (GDN_DEVERR_*).  Returns GDN_ERR_DEVICE if it
  * is nonzero, GDN_ERR_CUDA if the synchronisation failed, else GDN_OK.

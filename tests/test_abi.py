@@ -227,6 +227,28 @@ def test_conv_prefill_validation(L):
     assert call(a5=0, a7=0) == 0                # no sequences: nothing to do
 
 
+def test_cp_combine_validation(L):
+    f = L.gdn_cp_combine
+    # A_all, B_all, h0, R, rank, N, T_seg, HV, Dk, Dv, io, o, c, start, final, stream
+    base = [A, A + 4 * MB, None, 2, 1, 1, 100, 2, 128, 128, 1, A + 8 * MB, A + 9 * MB, A + 10 * MB, A + 11 * MB,
+            None]
+    def call(**kw):
+        a = list(base)
+        for i, val in kw.items():
+            a[int(i[1:])] = val
+        return f(*a)
+    assert call(a4=2) == 2                      # rank past R
+    assert call(a3=0) == 2                      # R
+    assert call(a8=64, a9=64) == 4              # d = 128 only
+    assert call(a0=None) == 1
+    assert call(a13=None) == 1                  # start state is required
+    assert call(a11=A + 8 * MB + 4) == 3        # o misaligned
+    assert call(a11=A + 9 * MB) == 5            # o over c
+    assert call(a13=A + 4 * MB) == 5            # start state over B_all
+    assert call(a14=A + 10 * MB) == 5           # final over start
+    assert call(a5=0) == 0                      # no sequences: nothing to do
+
+
 def test_decode_status_null(L):
     assert L.gdn_decode_status(None) == 1
     assert L.gdn_conv_status(None) == 1

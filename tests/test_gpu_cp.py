@@ -1,0 +1,64 @@
+"""Context-parallel prefill on one GPU with the ranks emulated one after another (no rank
+waits on another: the all-gather is a host-side stack): every segment through
+context_parallel.segment_transitions (two gdn_chunk_prefill runs), then gdn_cp_combine
+per segment; the outputs and final states against the oracle over the whole sequences."""
+import numpy as np
+import pytest
+
+from gated_deltanet_sequence_delta_b200 import inputs as I
+from harness import TOL, assert_close, gpu_gates, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(io, R, T_seg, N, HK, HV, seed):
+    import torch
+    import oracle
+    import gated_deltanet_sequence_delta_b200 as G
+    from gated_deltanet_sequence_delta_b200 import context_parallel as CP
+    T = R * T_seg
+    inp = I.make_prefill(N, T, HK, HV, 128, 128, io_dtype=io, seed=seed, h0_std=0.02)
+    q, k, v = to_dev(inp.q).view(N, T, HK, 128), to_dev(inp.k).view(N, T, HK, 128), to_dev(inp.v).view(N, T, HV, 128)
+    g, beta = gpu_gates(inp)
+    g, beta = g.view(N, T, HV), beta.view(N, T, HV)
+    h0 = to_dev(inp.h0)
+    parts = []
+    for r in range(R):
+        sl = slice(r * T_seg, (r + 1) * T_seg)
+        seg = [t[:, sl].contiguous() for t in (q, k, v, g, beta)]
+        parts.append(CP.segment_transitions(*seg, BT=inp.BT))
+    A_all = torch.stack([p[3] for p in parts])
+    B_all = torch.stack([p[1] for p in parts])
+    outs, finals, starts = [], [], []
+    for r in range(R):
+        o, _, c, _ = parts[r]
+        start, final = G.gdn_cp_combine(A_all, B_all, o, c, r, initial_state=h0)
+        outs.append(o)
+        finals.append(final)
+        starts.append(start)
+    o_cp = torch.cat(outs, dim=1)
+    # oracle over the whole sequences, on the same rounded inputs and the GPU's gates
+    o_ref, h_ref = oracle.recurrence(inp.q.f64().reshape(N, T, HK, 128), inp.k.f64().reshape(N, T, HK, 128),
+                                     inp.v.f64().reshape(N, T, HV, 128), to_np(g), to_np(beta),
+                                     h0=inp.h0.astype(np.float64))
+    tol = TOL[io]
+    assert_close(to_np(o_cp), o_ref, tol, f"context-parallel o ({io})", out_bf16=io == I.BF16)
+    for r in range(R):
+        assert_close(to_np(finals[r]), h_ref, tol, f"final state seen by rank {r}")
+    # every rank's start state is the state at its segment's first token
+    _, h_mid = oracle.recurrence(inp.q.f64().reshape(N, T, HK, 128)[:, :T_seg * 2],
+                                 inp.k.f64().reshape(N, T, HK, 128)[:, :T_seg * 2],
+                                 inp.v.f64().reshape(N, T, HV, 128)[:, :T_seg * 2], to_np(g)[:, :T_seg * 2],
+                                 to_np(beta)[:, :T_seg * 2], h0=inp.h0.astype(np.float64))
+    assert_close(to_np(starts[2]), h_mid, tol, "start state of segment 2")
+
+
+@pytest.mark.parametrize("io", [I.BF16, I.F32])
+def test_cp_four_segments_gqa(io):
+    """Four ragged segments of 200 tokens (not whole chunks), one sequence, HK=2, HV=4."""
+    _run(io, 4, 200, 1, 2, 4, 91)
+
+
+def test_cp_two_sequences():
+    """Two dense sequences, four segments of 256 tokens each, HK=HV=4, bf16."""
+    _run(I.BF16, 4, 256, 2, 4, 4, 92)
