@@ -285,7 +285,7 @@ struct PrepSmem {
     float X[3][16][17];
     float rk[64], rq[64], G[64], bt[64], bgr[64], red[8];
     float eu[64];   // rk_j exp(G_r - G_j), the token factor of the separated decays
-    float ga[2][64], ba[2][64];   // prefetched g, beta of the (up to two) value heads
+    float ga[2][64], ba[2][64];   // g, beta of value head gi in slot gi % 2, loaded ahead
     uint64_t bar_load, bar_v, bar_mma;
     uint32_t tmem_base;
 };
@@ -362,9 +362,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc::tma_load_3d(kq + 8192, &tm_q, &S.bar_load, 0, hk, si);
         tc::tma_load_3d(kq + 16384 + 8192, &tm_q, &S.bar_load, 64, hk, si);
     }
-    if (tid < 64) {   // gates of the group's value heads, prefetched under the TMA latency
+    if (tid < 64) {   // gates of the group's first two value heads, under the TMA latency
 #pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
+        for (int gi = 0; gi < (G < 2 ? G : 2); ++gi) {
             const int h = hk * G + gi;
             S.ga[gi][tid] = tid < cn ? g[(s + tid) * HV + h] : 0.f;
             S.ba[gi][tid] = tid < cn ? beta[(s + tid) * HV + h] : 0.f;
@@ -446,16 +446,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const bool last = gi == G - 1;
             // ---- running sum of the log-decays, write strengths -------------------------
             if (tid < 64) {
-                float gv = S.ga[gi][tid];
+                float gv = S.ga[gi & 1][tid];
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, gv, o);
                     if ((tid & 31) >= o) gv += y;
                 }
                 S.G[tid] = gv;
-                S.bt[tid] = S.ba[gi][tid];
+                S.bt[tid] = S.ba[gi & 1][tid];
             }
             __syncthreads();
+            if (G > 2 && gi + 2 < G && tid < 64) {   // slot gi % 2 is read: value head gi + 2's gates
+                S.ga[gi & 1][tid] = tid < cn ? g[(s + tid) * HV + h + 2] : 0.f;
+                S.ba[gi & 1][tid] = tid < cn ? beta[(s + tid) * HV + h + 2] : 0.f;
+            }
             if (tid >= 32 && tid < 64) S.G[tid] += S.G[31];
             __syncthreads();
             if (tid < 64) S.bgr[tid] = S.bt[tid] * expf(S.G[tid]);
@@ -1179,7 +1183,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank
 }
 
 bool prefill_tc_supported(int Dk, int Dv, int HK, int HV, int BT) {
-    return Dk == D && Dv == D && BT == C && (HV / HK == 1 || HV / HK == 2);
+    return Dk == D && Dv == D && BT == C && HV % HK == 0 && (HV / HK == 1 || HV / HK == 2 || HV / HK == 4);
 }
 
 size_t prefill_tc_workspace_bytes(int64_t n_tokens, int n_seqs, int HK, int HV) {
@@ -1259,27 +1263,20 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
     const int G = a.HV / a.HK;
     if (n_tokens > 0 && L.max_chunks > 0) {
         dim3 grid((unsigned)L.max_chunks, (unsigned)a.HK);
-        if (G == 1) {
-            e = cudaFuncSetAttribute(chunk_prep_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)kPrepSmemBytes);
-            if (e == cudaSuccess)   // four CTAs per SM need the largest shared-memory carveout
-                e = cudaFuncSetAttribute(chunk_prep_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                         (int)cudaSharedmemCarveoutMaxShared);
-            if (e != cudaSuccess) return e;
-            chunk_prep_kernel<1><<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T,
-                                                                 a.n_seqs, a.HV, a.scale, a.l2norm, a.HK, W, U, P,
-                                                                 QK, SC, a.status);
-        } else {
-            e = cudaFuncSetAttribute(chunk_prep_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)kPrepSmemBytes);
-            if (e == cudaSuccess)   // four CTAs per SM need the largest shared-memory carveout
-                e = cudaFuncSetAttribute(chunk_prep_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                         (int)cudaSharedmemCarveoutMaxShared);
-            if (e != cudaSuccess) return e;
-            chunk_prep_kernel<2><<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T,
-                                                                 a.n_seqs, a.HV, a.scale, a.l2norm, a.HK, W, U, P,
-                                                                 QK, SC, a.status);
-        }
+        auto launch_prep = [&](auto kern) -> cudaError_t {
+            cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)kPrepSmemBytes);
+            if (err == cudaSuccess)   // four CTAs per SM need the largest shared-memory carveout
+                err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                           (int)cudaSharedmemCarveoutMaxShared);
+            if (err != cudaSuccess) return err;
+            kern<<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T, a.n_seqs, a.HV,
+                                                   a.scale, a.l2norm, a.HK, W, U, P, QK, SC, a.status);
+            return cudaSuccess;
+        };
+        e = G == 1 ? launch_prep(chunk_prep_kernel<1>) : G == 2 ? launch_prep(chunk_prep_kernel<2>)
+                                                                 : launch_prep(chunk_prep_kernel<4>);
+        if (e != cudaSuccess) return e;
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         count_launch();

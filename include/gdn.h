@@ -129,7 +129,7 @@ GDN_API size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seq
  *                 not be shared by calls that may run concurrently.
  *   BT            chunk length: 64 (GDN_BF16) or 16, 32, 64 (GDN_F32).  BT only
  *                 changes rounding, never the result's definition.
- *                 GDN_BF16 with Dk = Dv = 128 and HV / HK in {1, 2} runs on the tensor
+ *                 GDN_BF16 with Dk = Dv = 128 and HV / HK in {1, 2, 4} runs on the tensor
  *                 cores (tcgen05); other GDN_BF16 shapes and GDN_F32 run on CUDA cores.
  *   scale         multiplies o (1.0 = the plain rule).
  *   qk_l2norm     nonzero: q and k rows are replaced by x / sqrt(sum x^2 + 1e-6)
@@ -162,7 +162,7 @@ GDN_API gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v
  *   norm_w  [Dv] fp32, shared by the value heads                                    (read)
  *   eps     >= 0 (the workloads' reading: 1e-6)
  * Other arguments as gdn_chunk_prefill, whose workspace size applies.  Only the
- * tensor-core configuration (bf16, Dk = Dv = 128, BT = 64, HV / HK in {1, 2}); others
+ * tensor-core configuration (bf16, Dk = Dv = 128, BT = 64, HV / HK in {1, 2, 4}); others
  * return UNSUPPORTED.  Errors: those of gdn_chunk_prefill, NULL (z or norm_w), SHAPE
  * (eps < 0 or NaN), ALIAS (o, final_state or workspace over z or norm_w).
  */

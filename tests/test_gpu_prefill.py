@@ -38,6 +38,19 @@ def test_varlen_small(io):
     check_prefill(inp)
 
 
+@pytest.mark.parametrize("packed", [False, True])
+def test_bf16_gqa_group4(packed):
+    """Four value heads per q/k head (HK=2, HV=8) on the tensor-core path: dense ragged or
+    packed sequences, with initial states."""
+    if packed:
+        lens = [70, 1, 191, 0, 64]
+        inp = I.make_prefill(1, int(sum(lens)), 2, 8, 128, 128, io_dtype=I.BF16, seed=12, h0_std=0.05,
+                             cu_seqlens=I.cu_from_lengths(lens))
+    else:
+        inp = I.make_prefill(2, 333, 2, 8, 128, 128, io_dtype=I.BF16, seed=12, h0_std=0.05)
+    check_prefill(inp)
+
+
 def test_stress_gates_small():
     """Forced resets (g = -20) and full writes (b = +20) at 1% each, T=4096."""
     inp = I.make_prefill(1, 4096, 4, 4, 128, 128, io_dtype=I.BF16, seed=10, h0_std=0.02,

@@ -37,6 +37,10 @@ def test_outgate_dense_ragged():
     _check(I.make_prefill(2, 333, 2, 4, 128, 128, io_dtype=I.BF16, seed=81, h0_std=0.05), 82)
 
 
+def test_outgate_gqa_group4():
+    _check(I.make_prefill(1, 200, 2, 8, 128, 128, io_dtype=I.BF16, seed=87, h0_std=0.05), 88)
+
+
 def test_outgate_mha_single_chunk_and_tail():
     _check(I.make_prefill(1, 70, 4, 4, 128, 128, io_dtype=I.BF16, seed=83, h0_std=0.05), 84)
 
