@@ -53,6 +53,9 @@ _SIGS = {
                          _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
     "gdn_conv_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_cp_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_cp_segment": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
+                        _i32, _f32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "gdn_cp_combine": ([_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _i32, _i32, ctypes.c_int, _vp, _vp, _vp, _vp,
                         _vp], ctypes.c_int),
     "gdn_decode_step_fused": ([_vp, ctypes.c_int, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_int, _vp, _vp, _vp,
@@ -370,6 +373,32 @@ def gdn_conv_prefill(x, conv_w, HK: int, HV: int, Dk: int = 128, Dv: int = 128, 
     return q, k, v, conv_state_out
 
 
+def gdn_cp_segment(q, k, v, g, beta, initial_state=None, cu_seqlens=None, BT: int = 64, scale: float = 1.0,
+                   qk_l2norm: bool = True, workspace=None):
+    """One rank's segment of a context-parallel prefill in one call (tensor-core shapes):
+    returns (o, final_state) of the segment's prefill and (c, A) of its transition run
+    (v = 0 from the identity), sharing one chunk-local stage."""
+    B_, T, HK, Dk = q.shape
+    HV, Dv = v.shape[-2:]
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B_
+    dcode = _dtype_code(q)
+    o = torch.empty((B_, T, HV, Dv), dtype=q.dtype, device=q.device)
+    c = torch.empty_like(o)
+    final_state = torch.empty((N, HV, Dk, Dv), dtype=torch.float32, device=q.device)
+    transition = torch.empty((N, HV, Dk, Dk), dtype=torch.float32, device=q.device)
+    need = prefill_workspace_bytes(B_ * T, N, HK, HV, Dk, Dv, BT, dcode)
+    if need == 0:
+        _check(4, "gdn_cp_segment")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().gdn_cp_segment(_ptr(q), _ptr(k), _ptr(v), dcode, _ptr(g), _ptr(beta), _ptr(initial_state),
+                              _ptr(cu_seqlens), B_, T, N, HK, HV, Dk, Dv, BT, float(scale), int(bool(qk_l2norm)),
+                              _ptr(o), _ptr(final_state), _ptr(c), _ptr(transition), _ptr(workspace),
+                              workspace.numel(), _stream())
+    _check(st, "gdn_cp_segment")
+    return o, final_state, c, transition
+
+
 def gdn_cp_combine(A_all, B_all, o, c, rank: int, initial_state=None, start_state=None, final_state=None,
                    output_final_state: bool = True):
     """The exchange step of a context-parallel prefill: A_all, B_all [R, N, HV, 128, 128]
@@ -390,6 +419,15 @@ def gdn_cp_combine(A_all, B_all, o, c, rank: int, initial_state=None, start_stat
                               _dtype_code(o), _ptr(o), _ptr(c), _ptr(start_state), _ptr(final_state), _stream())
     _check(st, "gdn_cp_combine")
     return start_state, final_state
+
+
+def gdn_cp_status() -> int:
+    """Synchronise the device, return gdn_cp_combine's error word and clear it."""
+    word = _i32(0)
+    st = lib().gdn_cp_status(ctypes.byref(word))
+    if st not in (0, 8):
+        _check(st, "gdn_cp_status")
+    return int(word.value)
 
 
 def gdn_conv_status() -> int:

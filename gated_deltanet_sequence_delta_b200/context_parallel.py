@@ -21,11 +21,17 @@ from . import binding as B
 def segment_transitions(q, k, v, g, beta, BT: int = 64, scale: float = 1.0, qk_l2norm: bool = True):
     """This rank's segment, dense [N, T_seg, ...] tensors on the GPU.  Returns (o0, Bs, c, As):
     o0 [N, T_seg, HV, Dv] and Bs [N, HV, Dk, Dv] from a zero start, c and As from the run
-    with v = 0 starting at the identity (Dk = Dv)."""
+    with v = 0 starting at the identity (Dk = Dv).  The tensor-core shapes take one call that
+    shares the chunk-local stage between the two runs; the others take two prefills."""
     N, _, _, Dk = q.shape
     HV, Dv = v.shape[-2:]
     if Dk != Dv:
         raise ValueError("context-parallel prefill needs Dk == Dv")
+    try:
+        return B.gdn_cp_segment(q, k, v, g, beta, BT=BT, scale=scale, qk_l2norm=qk_l2norm)
+    except B.GDNError as err:
+        if err.status != 4:   # anything but UNSUPPORTED is a real failure
+            raise
     o0, Bs = B.gdn_chunk_prefill(q, k, v, g, beta, BT=BT, scale=scale, qk_l2norm=qk_l2norm)
     eye = torch.eye(Dk, dtype=torch.float32, device=q.device).expand(N, HV, Dk, Dk).contiguous()
     c, As = B.gdn_chunk_prefill(q, k, torch.zeros_like(v), g, beta, initial_state=eye, BT=BT, scale=scale,

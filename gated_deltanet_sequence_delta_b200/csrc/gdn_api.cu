@@ -106,7 +106,8 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype i
                         const float* beta, const float* initial_state, const int32_t* cu_seqlens, int32_t B,
                         int64_t T, int32_t n_seqs, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
                         float scale, int32_t qk_l2norm, const void* z, const float* norm_w, float eps, void* o,
-                        float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+                        float* final_state, void* o_tr, float* final_tr, void* workspace, size_t workspace_bytes,
+                        void* stream) {
     // ---- sizes -----------------------------------------------------------------
     if (B < 0 || T < 0 || n_seqs < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || BT <= 0)
         return GDN_ERR_SHAPE;
@@ -128,9 +129,12 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype i
     if (workspace_bytes < need) return GDN_ERR_WORKSPACE;
     if (n_tok > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
     if (z && (!norm_w || !(eps >= 0.f))) return norm_w ? GDN_ERR_SHAPE : GDN_ERR_NULL;
-    if (z && !(io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT))) return GDN_ERR_UNSUPPORTED;
+    if ((z || o_tr) && !(io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT)))
+        return GDN_ERR_UNSUPPORTED;
+    if (o_tr && n_tok > 0 && !final_tr) return GDN_ERR_NULL;
     if (cu_seqlens == nullptr && n_tok == 0 && final_state == nullptr) return GDN_OK;
-    const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, workspace, z, norm_w};
+    const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, workspace, z, norm_w,
+                          o_tr, final_tr};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     // ---- aliasing ----------------------------------------------------------------
@@ -143,10 +147,15 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype i
     const Range ro{o, (size_t)n_tok * HV * Dv * es}, rhT{final_state, state_bytes};
     const Range rws{workspace, workspace_bytes};
     const Range rz{z, z ? (size_t)n_tok * HV * Dv * es : 0}, rnw{norm_w, z ? (size_t)Dv * 4 : 0};
-    for (Range out : {ro, rhT, rws}) {
+    const Range rotr{o_tr, o_tr ? (size_t)n_tok * HV * Dv * es : 0}, rhtr{final_tr, o_tr ? state_bytes : 0};
+    for (Range out : {ro, rhT, rws, rotr, rhtr}) {
         for (Range in : {rq, rk, rv, rg, rb, rcu, rz, rnw})
             if (overlap(out, in)) return GDN_ERR_ALIAS;
     }
+    for (Range tr : {rotr, rhtr})
+        for (Range other : {ro, rhT, rws, rh0})
+            if (overlap(tr, other)) return GDN_ERR_ALIAS;
+    if (overlap(rotr, rhtr)) return GDN_ERR_ALIAS;
     if (overlap(ro, rhT) || overlap(ro, rws) || overlap(rhT, rws) || overlap(ro, rh0) ||
         overlap(rws, rh0))
         return GDN_ERR_ALIAS;
@@ -167,6 +176,7 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype i
     a.T = T; a.n_seqs = n_seqs; a.HK = HK; a.HV = HV; a.Dk = Dk; a.Dv = Dv; a.BT = BT;
     a.scale = scale; a.l2norm = qk_l2norm ? 1 : 0; a.o = o; a.hT = final_state;
     a.z = z; a.norm_w = norm_w; a.eps = eps;
+    a.o_tr = o_tr; a.hT_tr = o_tr ? final_tr : nullptr;
     a.status = status;
     a.scratch = static_cast<char*>(workspace) + gdn::kStatusBytes;
     a.scratch_bytes = workspace_bytes - gdn::kStatusBytes;
@@ -184,7 +194,8 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dt
                              float scale, int32_t qk_l2norm, void* o, float* final_state,
                              void* workspace, size_t workspace_bytes, void* stream) {
     return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT,
-                        scale, qk_l2norm, nullptr, nullptr, 0.f, o, final_state, workspace, workspace_bytes, stream);
+                        scale, qk_l2norm, nullptr, nullptr, 0.f, o, final_state, nullptr, nullptr, workspace,
+                        workspace_bytes, stream);
 }
 
 gdn_status gdn_chunk_prefill_outgate(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
@@ -195,7 +206,20 @@ gdn_status gdn_chunk_prefill_outgate(const void* q, const void* k, const void* v
                                      float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
     if (!z) return GDN_ERR_NULL;
     return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT,
-                        scale, qk_l2norm, z, norm_w, eps, o, final_state, workspace, workspace_bytes, stream);
+                        scale, qk_l2norm, z, norm_w, eps, o, final_state, nullptr, nullptr, workspace,
+                        workspace_bytes, stream);
+}
+
+gdn_status gdn_cp_segment(const void* q, const void* k, const void* v, gdn_dtype io_dtype, const float* g,
+                          const float* beta, const float* initial_state, const int32_t* cu_seqlens, int32_t B,
+                          int64_t T, int32_t n_seqs, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
+                          float scale, int32_t qk_l2norm, void* o, float* final_state, void* c, float* transition,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    if (!c) return GDN_ERR_NULL;
+    if (Dk != Dv) return GDN_ERR_UNSUPPORTED;
+    return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT,
+                        scale, qk_l2norm, nullptr, nullptr, 0.f, o, final_state, c, transition, workspace,
+                        workspace_bytes, stream);
 }
 
 gdn_status gdn_chunk_prefill_status(const void* workspace, void* stream, int32_t* device_error) {
@@ -348,6 +372,17 @@ gdn_status gdn_cp_combine(const float* A_all, const float* B_all, const float* i
     return cuda_status(gdn::launch_cp_combine(A_all, B_all, initial_state, R, rank, n_seqs, T_seg, HV,
                                               io_dtype == GDN_BF16, o, c, start_state, final_state,
                                               (cudaStream_t)stream));
+}
+
+gdn_status gdn_cp_status(int32_t* device_error) {
+    if (!device_error) return GDN_ERR_NULL;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e);
+    int32_t word = 0;
+    e = gdn::read_cp_error(&word, true);
+    if (e != cudaSuccess) return cuda_status(e);
+    *device_error = word;
+    return word ? GDN_ERR_DEVICE : GDN_OK;
 }
 
 gdn_status gdn_conv_status(int32_t* device_error) {

@@ -118,6 +118,10 @@ cudaError_t launch_cp_combine(const float* A_all, const float* B_all, const floa
                               int64_t T_seg, int HV, bool bf16, void* o, const void* c, float* start_state,
                               float* final_state, cudaStream_t s);
 
+// Read (and on request clear) the device word the tensor-core correction of gdn_cp_combine sets
+// on a timeout.
+cudaError_t read_cp_error(int32_t* out, bool reset);
+
 // Read (and on request clear) the device word the bf16 convolution kernel sets on a timeout.
 cudaError_t read_conv_error(int32_t* out, bool reset);
 
@@ -142,6 +146,8 @@ struct PrefillArgs {
     const void* z;            // output epilogue gate inputs [.., HV, Dv] io dtype, or null (none)
     const float* norm_w;      // output epilogue norm weights [Dv] (with z)
     float eps;                // output epilogue norm epsilon (with z)
+    void* o_tr;               // with hT_tr: the transition run's outputs (v = 0 from the identity;
+    float* hT_tr;             //   tensor-core path only), or null
     int32_t* status;          // device status word (workspace)
     void* scratch;            // workspace after the status words
     size_t scratch_bytes;
@@ -151,7 +157,7 @@ cudaError_t launch_check_cu_seqlens(const int32_t* cu, int n_seqs, int64_t T, in
                                     cudaStream_t s);
 cudaError_t launch_prefill_cudacore(const PrefillArgs& a, cudaStream_t s);
 
-// Tensor-core (tcgen05) prefill: bf16, Dk = Dv = 128, BT = 64, HV / HK in {1, 2}.
+// Tensor-core (tcgen05) prefill: bf16, Dk = Dv = 128, BT = 64, HV / HK in {1, 2, 4}.
 bool prefill_tc_supported(int Dk, int Dv, int HK, int HV, int BT);
 size_t prefill_tc_workspace_bytes(int64_t n_tokens, int n_seqs, int HK, int HV);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_t s);

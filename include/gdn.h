@@ -221,6 +221,25 @@ GDN_API gdn_status gdn_conv_prefill(const void* x, gdn_dtype io_dtype, const flo
 GDN_API gdn_status gdn_conv_status(int32_t* device_error);
 
 /*
+ * gdn_cp_segment -- one rank's work on its segment in a context-parallel prefill (see
+ * gdn_cp_combine): the segment's gdn_chunk_prefill (o, final_state, from initial_state or
+ * zero) and, on the same chunk-local stage, its transition run (v = 0 from the identity):
+ *   c          [B, T, HV, Dv] io_dtype: c_t = scale A_{<=t}^T q_t                   (written)
+ *   transition [n_seqs, HV, Dk, Dk] fp32: A, the product of the segment's transitions
+ *                                                                                   (written)
+ * The other arguments and the errors are those of gdn_chunk_prefill; only the tensor-core
+ * configuration (bf16, Dk = Dv = 128, BT = 64, HV / HK in {1, 2, 4}) is supported (others:
+ * UNSUPPORTED; two gdn_chunk_prefill calls give the same results).  c and transition may
+ * not overlap any other buffer.
+ */
+GDN_API gdn_status gdn_cp_segment(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                                  const float* g, const float* beta, const float* initial_state,
+                                  const int32_t* cu_seqlens, int32_t B, int64_t T, int32_t n_seqs,
+                                  int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT, float scale,
+                                  int32_t qk_l2norm, void* o, float* final_state, void* c,
+                                  float* transition, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * gdn_cp_combine -- the exchange step of a context-parallel prefill, in which each of R
  * ranks holds one consecutive segment of the same sequences (rank r the r-th segment of
  * T_seg tokens).  Over a segment the rule is affine in the state it starts from (the
@@ -237,13 +256,23 @@ GDN_API gdn_status gdn_conv_status(int32_t* device_error);
  *   c             [n_seqs, T_seg, HV, 128] io_dtype                              (read)
  *   start_state   [n_seqs, HV, 128, 128] fp32, H_start of this rank's segment   (written)
  *   final_state   [n_seqs, HV, 128, 128] fp32, the state after segment R - 1, or NULL
- * Dk = Dv = 128 only.  No output may overlap an input or another output.
+ * Dk = Dv = 128 only.  No output may overlap an input or another output.  For bf16 the
+ * correction runs on the tensor cores (H_start rounded to bf16 for the product) with
+ * bounded waits; a wait that expires (no such case is known) records GDN_DEVERR_TIMEOUT,
+ * which gdn_cp_status reports.
  * Errors: NULL, SHAPE (R, rank, sizes), ALIGN, UNSUPPORTED, ALIAS, CUDA.
  */
 GDN_API gdn_status gdn_cp_combine(const float* A_all, const float* B_all, const float* initial_state,
                                   int32_t R, int32_t rank, int32_t n_seqs, int64_t T_seg, int32_t HV,
                                   int32_t Dk, int32_t Dv, gdn_dtype io_dtype, void* o, const void* c,
                                   float* start_state, float* final_state, void* stream);
+
+/*
+ * Synchronises the device, then reads and clears the device word of gdn_cp_combine's
+ * tensor-core correction (GDN_DEVERR_NONE or GDN_DEVERR_TIMEOUT) into *device_error.
+ * Returns GDN_ERR_DEVICE if it is nonzero.  Errors: NULL, CUDA.
+ */
+GDN_API gdn_status gdn_cp_status(int32_t* device_error);
 
 /*
  * Synchronises `stream`, then reads the device status word of a prefill

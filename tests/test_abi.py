@@ -93,6 +93,29 @@ def test_prefill_outgate_validation(L):
     assert _prefill_outgate(L, N=0, B=0) == 0              # nothing to do
 
 
+def _cp_segment(L, **kw):
+    args = dict(q=A, k=A + 64 * MB, v=A + 128 * MB, io=1, g=A + 192 * MB, beta=A + 200 * MB,
+                h0=None, cu=None, B=1, T=128, N=1, HK=2, HV=4, Dk=128, Dv=128, BT=64, scale=1.0,
+                l2=1, o=A + 256 * MB, hT=A + 384 * MB, c=A + 512 * MB, tr=A + 600 * MB,
+                ws=A + 448 * MB, ws_bytes=1 << 20)
+    args.update(kw)
+    return L.gdn_cp_segment(args["q"], args["k"], args["v"], args["io"], args["g"], args["beta"], args["h0"],
+                            args["cu"], args["B"], args["T"], args["N"], args["HK"], args["HV"], args["Dk"],
+                            args["Dv"], args["BT"], args["scale"], args["l2"], args["o"], args["hT"], args["c"],
+                            args["tr"], args["ws"], args["ws_bytes"], None)
+
+
+def test_cp_segment_validation(L):
+    assert _cp_segment(L, c=None) == 1
+    assert _cp_segment(L, tr=None) == 1                   # the transition output is required
+    assert _cp_segment(L, Dv=64) == 4                     # Dk == Dv only
+    assert _cp_segment(L, io=0, BT=64) == 4               # fp32: no tensor-core path
+    assert _cp_segment(L, HV=6, HK=2) == 4                # GQA group 3
+    assert _cp_segment(L, c=A + 256 * MB + 64) == 5       # c over o
+    assert _cp_segment(L, tr=A + 384 * MB) == 5           # transition over the final state
+    assert _cp_segment(L, N=0, B=0) == 0                  # nothing to do
+
+
 def test_prefill_workspace_query(L):
     assert L.gdn_chunk_prefill_workspace_bytes(32768, 1, 16, 32, 128, 128, 64, 1) >= 256
     assert L.gdn_chunk_prefill_workspace_bytes(256, 1, 2, 2, 64, 64, 64, 0) >= 256
@@ -252,6 +275,7 @@ def test_cp_combine_validation(L):
 def test_decode_status_null(L):
     assert L.gdn_decode_status(None) == 1
     assert L.gdn_conv_status(None) == 1
+    assert L.gdn_cp_status(None) == 1
 
 
 def test_missing_library_fails_loudly(tmp_path):

@@ -51,6 +51,7 @@ def _run(io, R, T_seg, N, HK, HV, seed):
                                  inp.v.f64().reshape(N, T, HV, 128)[:, :T_seg * 2], to_np(g)[:, :T_seg * 2],
                                  to_np(beta)[:, :T_seg * 2], h0=inp.h0.astype(np.float64))
     assert_close(to_np(starts[2]), h_mid, tol, "start state of segment 2")
+    assert G.gdn_cp_status() == 0
 
 
 @pytest.mark.parametrize("io", [I.BF16, I.F32])
@@ -62,3 +63,22 @@ def test_cp_four_segments_gqa(io):
 def test_cp_two_sequences():
     """Two dense sequences, four segments of 256 tokens each, HK=HV=4, bf16."""
     _run(I.BF16, 4, 256, 2, 4, 4, 92)
+
+
+def test_cp_segment_matches_two_prefills():
+    """gdn_cp_segment (one chunk-local stage, two carries) against gdn_chunk_prefill from
+    zero (o, final state: bit for bit) and gdn_chunk_prefill with v = 0 from the identity
+    (c, A: to the usual tolerance; the fp16 data scale of the two carries may differ)."""
+    import torch
+    import gated_deltanet_sequence_delta_b200 as G
+    inp = I.make_prefill(2, 300, 2, 4, 128, 128, io_dtype=I.BF16, seed=93)
+    q, k, v = to_dev(inp.q).view(2, 300, 2, 128), to_dev(inp.k).view(2, 300, 2, 128), to_dev(inp.v).view(2, 300, 4, 128)
+    g, beta = gpu_gates(inp)
+    g, beta = g.view(2, 300, 4), beta.view(2, 300, 4)
+    o, hT, c, A = G.gdn_cp_segment(q, k, v, g, beta)
+    o2, hT2 = G.gdn_chunk_prefill(q, k, v, g, beta)
+    eye = torch.eye(128, dtype=torch.float32, device="cuda").expand(2, 4, 128, 128).contiguous()
+    c2, A2 = G.gdn_chunk_prefill(q, k, torch.zeros_like(v), g, beta, initial_state=eye)
+    assert torch.equal(o, o2) and torch.equal(hT, hT2)
+    assert_close(to_np(c), to_np(c2), TOL[I.BF16], "c", out_bf16=True)
+    assert_close(to_np(A), to_np(A2), TOL[I.BF16], "A")
