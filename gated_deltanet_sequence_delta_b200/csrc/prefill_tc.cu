@@ -750,7 +750,9 @@ __device__ __forceinline__ void store_op_row(f16* op, int k, const float* v, flo
 // on the serial chain: the producer streams each chunk's z tile and row scalars into a
 // ring of NZ slots, D_a and D_c rotate over three buffers, and the MMA warp reuses a
 // buffer only after the output warps release it (ofree).
-template <bool OUTG>
+// TR: the transition run of a context-parallel segment: U taken as zero (v = 0) and the
+// identity as the initial state (Dk = Dv), on the chunk-local operands of the same call.
+template <bool OUTG, bool TR = false>
 __global__ void __launch_bounds__(carry_threads(OUTG), 1)
 chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qk,
                    const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_u,
@@ -759,7 +761,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                    const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HK, int HV,
                    const float* __restrict__ h0, float* __restrict__ hT, bf16* __restrict__ o,
                    const bf16* __restrict__ zg, const float* __restrict__ norm_w, float eps,
-                   int32_t* __restrict__ status, int zero_u, int ident_h0) {
+                   int32_t* __restrict__ status) {
     constexpr int nb = OUTG ? 3 : 2;   // buffers of D_a and D_c
     extern __shared__ uint8_t smem_raw[];
     CarrySmem& S = *reinterpret_cast<CarrySmem*>(align1024(smem_raw));
@@ -917,8 +919,8 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         const size_t hrow = (((size_t)n * HV + h) * D + t) * D + vs * NS;
         float m = 0.f;
 #pragma unroll
-        for (int j = 0; j < NS; ++j) {   // the initial state (ident_h0: the identity, Dk = Dv)
-            Hr[j] = ident_h0 ? (t == vs * NS + j ? 1.f : 0.f) : (h0 ? h0[hrow + j] : 0.f);
+        for (int j = 0; j < NS; ++j) {   // the initial state (TR: the identity)
+            Hr[j] = TR ? (t == vs * NS + j ? 1.f : 0.f) : (h0 ? h0[hrow + j] : 0.f);
             m = fmaxf(m, fabsf(Hr[j]));
         }
         // data scale: fp16 operands carry x * sc with sc = 2^-e, max(|h0|, |v|) * sc < 1
@@ -979,7 +981,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 float x[NS];
                 tc::tmem_ld32(tA + (uint32_t)(c % nb) * 32 + lane_base, x);
                 tc::tmem_wait_ld();
-                const float dr = B.SC[64 + t], uinv = zero_u ? 0.f : B.SC[SC_UINV];   // zero_u: v = 0
+                const float dr = B.SC[64 + t], uinv = TR ? 0.f : B.SC[SC_UINV];   // TR: v = 0
                 const uint4* urow = reinterpret_cast<const uint4*>(B.U + t * NS);
                 float dv[NS];
 #pragma unroll
@@ -1288,14 +1290,17 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
         if (e != cudaSuccess) return e;
         chunk_carry_kernel<false><<<blocks, carry_threads(false), kCarrySmemBytes, s>>>(
             tw, tqk, tp, tu, tw, SC, a.cu, chunk_off, a.T, a.n_seqs, a.HK, a.HV, a.h0, a.hT, (bf16*)a.o, nullptr,
-            nullptr, 0.f, a.status, 0, 0);
+            nullptr, 0.f, a.status);
         if (a.o_tr) {   // the transition run on the same chunk-local operands: v = 0 from the identity
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;
             count_launch();
-            chunk_carry_kernel<false><<<blocks, carry_threads(false), kCarrySmemBytes, s>>>(
+            e = cudaFuncSetAttribute(chunk_carry_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kCarrySmemBytes);
+            if (e != cudaSuccess) return e;
+            chunk_carry_kernel<false, true><<<blocks, carry_threads(false), kCarrySmemBytes, s>>>(
                 tw, tqk, tp, tu, tw, SC, a.cu, chunk_off, a.T, a.n_seqs, a.HK, a.HV, nullptr, a.hT_tr,
-                (bf16*)a.o_tr, nullptr, nullptr, 0.f, a.status, 1, 1);
+                (bf16*)a.o_tr, nullptr, nullptr, 0.f, a.status);
         }
     } else {   // the head's four column slices as one cluster (output epilogue)
         // z [tokens, HV, Dv] bf16: one slice's 32 values of one head for 64 tokens per tile
@@ -1322,7 +1327,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, chunk_carry_kernel<true>, tw, tqk, tp, tu, tz, (const float*)SC, a.cu,
                                (const int32_t*)chunk_off, a.T, a.n_seqs, a.HK, a.HV, a.h0, a.hT, (bf16*)a.o,
-                               (const bf16*)a.z, a.norm_w, a.eps, a.status, 0, 0);
+                               (const bf16*)a.z, a.norm_w, a.eps, a.status);
         if (e != cudaSuccess) return e;
     }
     e = cudaGetLastError();
