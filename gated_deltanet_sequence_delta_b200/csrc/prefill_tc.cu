@@ -354,6 +354,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int si = (int)s;
     uint8_t* kq = reinterpret_cast<uint8_t*>(&S.KQ[0][0]);
     uint32_t mma_phase = 0;
+    int v_loads = 0;   // V tile copies issued (thread 0)
 
     if (tid == 0) {
         tc::mbar_expect_tx(&S.bar_load, 4 * 64 * 64 * 2);
@@ -436,6 +437,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         __syncthreads();
         if (tid == 0) {   // Q is consumed: its rows now receive V of the first value head
             tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+            ++v_loads;
             tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, hk * G, si);
             tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, hk * G, si);
         }
@@ -629,6 +631,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc::tc_fence_after();
                 if (tid == 0) {   // the V rows are free again: next head's V
                     tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+                    ++v_loads;
                     tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, h + 1, si);
                     tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, h + 1, si);
                 }
@@ -643,7 +646,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0) tc::tmem_dealloc(tmem, kPrepTmemCols);
     return;
 abort:
-    if (tid == 0) record_timeout(status);
+    if (tid == 0) {
+        record_timeout(status);
+        // the copies and products still in flight land before the shared memory and TMEM are
+        // released; each wait is for the latest phase of its barrier (at once if complete)
+        (void)tc::mbar_wait(&S.bar_load, 0, 50000000ull);
+        if (v_loads > 0) (void)tc::mbar_wait(&S.bar_v, (uint32_t)((v_loads - 1) & 1), 50000000ull);
+        (void)tc::mbar_wait(&S.bar_mma, mma_phase ^ 1u, 50000000ull);
+    }
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kPrepTmemCols);
