@@ -355,6 +355,10 @@ gdn_status gdn_cp_combine(const float* A_all, const float* B_all, const float* i
                           void* stream) {
     if (R < 1 || rank < 0 || rank >= R || n_seqs < 0 || T_seg < 0 || HV <= 0) return GDN_ERR_SHAPE;
     if (!dtype_ok(io_dtype) || Dk != 128 || Dv != 128) return GDN_ERR_UNSUPPORTED;
+    // sizes the correction kernels address: 128-token tiles as a grid row (fp32), 32-bit tile
+    // coordinates (bf16)
+    if (io_dtype == GDN_F32 ? (T_seg + 127) / 128 > 65535 : (int64_t)n_seqs * T_seg > INT32_MAX - 128)
+        return GDN_ERR_UNSUPPORTED;
     if (n_seqs == 0) return GDN_OK;
     if (!A_all || !B_all || !start_state || (T_seg > 0 && (!o || !c))) return GDN_ERR_NULL;
     const void* ptrs[] = {A_all, B_all, initial_state, o, c, start_state, final_state};

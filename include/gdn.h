@@ -256,7 +256,8 @@ GDN_API gdn_status gdn_cp_segment(const void* q, const void* k, const void* v, g
  *   c             [n_seqs, T_seg, HV, 128] io_dtype                              (read)
  *   start_state   [n_seqs, HV, 128, 128] fp32, H_start of this rank's segment   (written)
  *   final_state   [n_seqs, HV, 128, 128] fp32, the state after segment R - 1, or NULL
- * Dk = Dv = 128 only.  No output may overlap an input or another output.  For bf16 the
+ * Dk = Dv = 128 only; up to 65535 x 128 tokens per segment (fp32) or 2^31 - 129 tokens over
+ * all sequences (bf16).  No output may overlap an input or another output.  For bf16 the
  * correction runs on the tensor cores (H_start rounded to bf16 for the product) with
  * bounded waits; a wait that expires (no such case is known) records GDN_DEVERR_TIMEOUT,
  * which gdn_cp_status reports.

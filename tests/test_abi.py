@@ -269,6 +269,8 @@ def test_cp_combine_validation(L):
     assert call(a11=A + 9 * MB) == 5            # o over c
     assert call(a13=A + 4 * MB) == 5            # start state over B_all
     assert call(a14=A + 10 * MB) == 5           # final over start
+    assert call(a10=0, a6=65535 * 128 + 1) == 4  # fp32: more token tiles than a grid row holds
+    assert call(a5=2, a6=(1 << 30)) == 4         # bf16: past 32-bit tile coordinates
     assert call(a5=0) == 0                      # no sequences: nothing to do
 
 
