@@ -8,7 +8,8 @@ library.
 _BINDING = ("gdn_gates", "gdn_chunk_prefill", "gdn_chunk_prefill_outgate", "gdn_chunk_prefill_status",
             "gdn_conv_prefill", "gdn_conv_status", "gdn_cp_segment", "gdn_cp_combine", "gdn_cp_status", "gdn_decode_step", "gdn_decode_step_gated", "gdn_decode_step_fused",
             "gdn_decode_status", "gdn_chunk_prefill_host", "prefill_host_workspace_bytes",
-            "GDNError", "GDNLibraryError", "prefill_workspace_bytes", "kernel_launches")
+            "GDNError", "GDNLibraryError", "prefill_workspace_bytes", "kernel_launches", "testing_stall",
+            "STALL_NONE", "STALL_DECODE", "STALL_PREFILL_PREP")
 
 __all__ = list(_BINDING)
 

@@ -52,6 +52,7 @@ _SIGS = {
     "gdn_decode_step": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                          _f32, _i32, _vp, _vp], ctypes.c_int),
     "gdn_decode_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_testing_stall": ([_i32], ctypes.c_int),
     "gdn_conv_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
     "gdn_cp_status": ([ctypes.POINTER(_i32)], ctypes.c_int),
     "gdn_cp_segment": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
@@ -446,3 +447,12 @@ def gdn_decode_status() -> int:
     if st not in (0, 8):
         _check(st, "gdn_decode_status")
     return int(word.value)
+
+
+STALL_NONE, STALL_DECODE, STALL_PREFILL_PREP = 0, 1, 2
+
+
+def testing_stall(site: int):
+    """Test hook: make one CTA of the chosen kernel wait for copies that are never issued,
+    so that its bounded wait runs out (STALL_NONE restores normal operation)."""
+    _check(lib().gdn_testing_stall(int(site)), "gdn_testing_stall")

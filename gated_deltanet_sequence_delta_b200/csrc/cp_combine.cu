@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(128) cp_correct_tc_kernel(const __grid_constan
     tc::fence_async_smem();
     int issued = mine < 2 ? mine : 2;   // tiles whose copies thread 0 has started
     int landed = 0;                     // tiles whose copies completed and were waited for
+    int products = 0;                   // MMA groups thread 0 has committed to bar_mma
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     for (int i = 0; i < mine; ++i) {
         const int st = i & 1;
@@ -239,6 +240,7 @@ __global__ void __launch_bounds__(128) cp_correct_tc_kernel(const __grid_constan
                              tc::idesc_bf16(128, 128, 0, 0), kk > 0);
             }
             tc::mma_commit(&S.bar_mma);
+            ++products;
         }
         ok = tc::mbar_wait(&S.bar_mma, (uint32_t)(i & 1));
         tc::tc_fence_after();
@@ -275,9 +277,13 @@ __global__ void __launch_bounds__(128) cp_correct_tc_kernel(const __grid_constan
             break;
         }
     }
-    if (tid == 0)   // copies started but never waited for (a wait gave up) land before the CTA leaves;
-                    // each is the latest use of its stage, so its parity is the one still pending
+    if (tid == 0) {   // copies started but never waited for (a wait gave up) land before the CTA leaves;
+                      // each is the latest use of its stage, so its parity is the one still pending
         for (int i = landed; i < issued; ++i) (void)tc::mbar_wait(&S.full[i & 1], (uint32_t)((i >> 1) & 1), 50000000ull);
+        // so does the latest MMA group, which may still read the tiles and write TMEM (at once
+        // if it completed)
+        if (products > 0) (void)tc::mbar_wait(&S.bar_mma, (uint32_t)((products - 1) & 1), 50000000ull);
+    }
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, 128);

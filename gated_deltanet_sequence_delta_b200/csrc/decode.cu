@@ -194,7 +194,7 @@ template <typename IO, bool CONV>
 __global__ void __launch_bounds__(kSThreads, 1)
 decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                      const DecodeConv conv, const DecodeGates gates, float* __restrict__ state, int n_items,
-                     int HK, int HV, float scale, int l2norm, IO* __restrict__ o) {
+                     int HK, int HV, float scale, int l2norm, IO* __restrict__ o, int stall) {
     using QT = typename std::conditional<CONV, float, IO>::type;   // element type of the q, k, v rows
     constexpr int CPL = kSD / 32;   // 4 columns per lane
     constexpr uint32_t kRowBytes = kSD * sizeof(IO);
@@ -223,6 +223,9 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
                     atomicExch(&g_decode_error, GDN_DEVERR_TIMEOUT);
                     break;
                 }
+                // test hook (gdn_testing_stall): the first CTA's first item gets no copies, so
+                // the compute warps' wait for it runs out
+                if (stall && blockIdx.x == 0 && i == 0) continue;
                 const int bh = blockIdx.x + i * G;
                 const int b = bh / HV, h = bh - b * HV, hk = h / (HV / HK);
                 StagedSlot& B = S.st[st];
@@ -403,7 +406,8 @@ cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, co
     if (e != cudaSuccess) return e;
     const int grid = n_items < sms ? n_items : sms;
     decode_staged_kernel<IO, CONV><<<grid, kSThreads, smem, s>>>(
-        (const IO*)q, (const IO*)k, (const IO*)v, conv, gates, state, n_items, HK, HV, scale, l2norm, (IO*)o);
+        (const IO*)q, (const IO*)k, (const IO*)v, conv, gates, state, n_items, HK, HV, scale, l2norm, (IO*)o,
+        testing_stall_site() == GDN_STALL_DECODE ? 1 : 0);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;

@@ -11,6 +11,7 @@ namespace {
 
 thread_local int g_last_cuda_error = 0;
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_stall_site{0};   // gdn_testing_stall
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -39,6 +40,7 @@ gdn_status cuda_status(cudaError_t e) {
 
 namespace gdn {
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+int testing_stall_site() { return g_stall_site.load(std::memory_order_relaxed); }
 }  // namespace gdn
 
 extern "C" {
@@ -61,6 +63,12 @@ const char* gdn_status_string(int status) {
 }
 
 int gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+gdn_status gdn_testing_stall(int32_t site) {
+    if (site < GDN_STALL_NONE || site > GDN_STALL_PREFILL_PREP) return GDN_ERR_SHAPE;
+    g_stall_site.store(site, std::memory_order_relaxed);
+    return GDN_OK;
+}
 
 int gdn_last_cuda_error(void) { return g_last_cuda_error; }
 
@@ -100,6 +108,28 @@ size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seqs, int32
 
 }  // extern "C"
 
+namespace gdn {
+// The size checks of gdn_chunk_prefill, in its order: SHAPE for sizes out of range or
+// inconsistent with the layout, UNSUPPORTED for head dims, chunk sizes or dtypes that no
+// kernel takes (including sizes past the tile-copy coordinates); GDN_OK otherwise.
+gdn_status prefill_check_sizes(gdn_dtype io_dtype, bool packed, int32_t B, int64_t T, int32_t n_seqs, int32_t HK,
+                               int32_t HV, int32_t Dk, int32_t Dv, int32_t BT) {
+    if (B < 0 || T < 0 || n_seqs < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || BT <= 0)
+        return GDN_ERR_SHAPE;
+    if (HV % HK != 0) return GDN_ERR_SHAPE;
+    if (packed) {
+        if (B != 1) return GDN_ERR_SHAPE;
+        if (T > INT32_MAX) return GDN_ERR_SHAPE;
+    } else if (n_seqs != B) {
+        return GDN_ERR_SHAPE;
+    }
+    if (!dtype_ok(io_dtype) || !head_dim_ok(Dk) || !head_dim_ok(Dv)) return GDN_ERR_UNSUPPORTED;
+    if (gdn_chunk_prefill_workspace_bytes((int64_t)B * T, n_seqs, HK, HV, Dk, Dv, BT, io_dtype) == 0)
+        return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+}  // namespace gdn
+
 namespace {
 // gdn_chunk_prefill, with the output epilogue when z is given (tensor-core path only)
 gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype io_dtype, const float* g,
@@ -109,19 +139,11 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype i
                         float* final_state, void* o_tr, float* final_tr, void* workspace, size_t workspace_bytes,
                         void* stream) {
     // ---- sizes -----------------------------------------------------------------
-    if (B < 0 || T < 0 || n_seqs < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || BT <= 0)
-        return GDN_ERR_SHAPE;
-    if (HV % HK != 0) return GDN_ERR_SHAPE;
-    if (cu_seqlens) {
-        if (B != 1) return GDN_ERR_SHAPE;
-        if (T > INT32_MAX) return GDN_ERR_SHAPE;
-    } else if (n_seqs != B) {
-        return GDN_ERR_SHAPE;
-    }
-    if (!dtype_ok(io_dtype) || !head_dim_ok(Dk) || !head_dim_ok(Dv)) return GDN_ERR_UNSUPPORTED;
+    const gdn_status sz =
+        gdn::prefill_check_sizes(io_dtype, cu_seqlens != nullptr, B, T, n_seqs, HK, HV, Dk, Dv, BT);
+    if (sz != GDN_OK) return sz;
     const size_t need = gdn_chunk_prefill_workspace_bytes((int64_t)B * T, n_seqs, HK, HV, Dk, Dv,
                                                           BT, io_dtype);
-    if (need == 0) return GDN_ERR_UNSUPPORTED;
     const int64_t n_tok = (int64_t)B * T;
     if (n_seqs == 0) return GDN_OK;
     // ---- pointers ----------------------------------------------------------------

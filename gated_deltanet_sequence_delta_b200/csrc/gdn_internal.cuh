@@ -47,6 +47,10 @@ __device__ __forceinline__ float l2_inv(float sumsq, int enabled) {
 // Launch accounting: every launcher calls count_launch() after a successful launch.
 void count_launch(int n = 1);
 
+// The site gdn_testing_stall selected (GDN_STALL_NONE normally); launchers read it on the
+// host and pass the kernels a flag.
+int testing_stall_site();
+
 // Workspace layout: [0, 256) status words; then kernel-specific scratch.
 constexpr size_t kStatusBytes = 256;
 
@@ -152,6 +156,11 @@ struct PrefillArgs {
     void* scratch;            // workspace after the status words
     size_t scratch_bytes;
 };
+
+// The size checks of gdn_chunk_prefill (GDN_OK, GDN_ERR_SHAPE or GDN_ERR_UNSUPPORTED), shared
+// by every prefill entry point so that they reject the same sizes with the same status.
+gdn_status prefill_check_sizes(gdn_dtype io_dtype, bool packed, int32_t B, int64_t T, int32_t n_seqs, int32_t HK,
+                               int32_t HV, int32_t Dk, int32_t Dv, int32_t BT);
 
 cudaError_t launch_check_cu_seqlens(const int32_t* cu, int n_seqs, int64_t T, int32_t* status,
                                     cudaStream_t s);

@@ -322,7 +322,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const float* __restrict__ beta, const int32_t* __restrict__ cu,
                   const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HV, float scale,
                   int l2norm, int HK, f16* __restrict__ Wg, f16* __restrict__ Ug, f16* __restrict__ Pg,
-                  f16* __restrict__ QKg, float* __restrict__ SCg, int32_t* __restrict__ status) {
+                  f16* __restrict__ QKg, float* __restrict__ SCg, int32_t* __restrict__ status, int stall) {
     extern __shared__ uint8_t smem_raw[];
     PrepSmem& S = *reinterpret_cast<PrepSmem*>(align1024(smem_raw));
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -435,7 +435,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         tc::fence_async_smem();
         __syncthreads();
-        if (tid == 0) {   // Q is consumed: its rows now receive V of the first value head
+        // Q is consumed: its rows now receive V of the first value head (test hook,
+        // gdn_testing_stall: not for the first CTA, whose wait for it then runs out)
+        if (tid == 0 && !(stall && chunk == 0 && hk == 0)) {
             tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
             ++v_loads;
             tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, hk * G, si);
@@ -1283,7 +1285,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
                                            (int)cudaSharedmemCarveoutMaxShared);
             if (err != cudaSuccess) return err;
             kern<<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T, a.n_seqs, a.HV,
-                                                   a.scale, a.l2norm, a.HK, W, U, P, QK, SC, a.status);
+                                                   a.scale, a.l2norm, a.HK, W, U, P, QK, SC, a.status,
+                                                   testing_stall_site() == GDN_STALL_PREFILL_PREP ? 1 : 0);
             return cudaSuccess;
         };
         e = G == 1 ? launch_prep(chunk_prep_kernel<1>) : G == 2 ? launch_prep(chunk_prep_kernel<2>)

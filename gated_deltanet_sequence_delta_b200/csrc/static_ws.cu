@@ -51,10 +51,12 @@ extern "C" gdn_status gdn_chunk_prefill_static_ws(
     const float* initial_state, const int32_t* cu_seqlens, int32_t B, int64_t T, int32_t n_seqs, int32_t HK,
     int32_t HV, int32_t Dk, int32_t Dv, int32_t BT, float scale, int32_t qk_l2norm, void* o, float* final_state,
     void* stream) {
-    if (B < 0 || T < 0 || n_seqs < 0) return GDN_ERR_SHAPE;
+    // the sizes are checked as gdn_chunk_prefill checks them, so both return the same status
+    const gdn_status sz =
+        gdn::prefill_check_sizes(io_dtype, cu_seqlens != nullptr, B, T, n_seqs, HK, HV, Dk, Dv, BT);
+    if (sz != GDN_OK) return sz;
     const size_t need =
         gdn_chunk_prefill_workspace_bytes((int64_t)B * T, n_seqs, HK, HV, Dk, Dv, BT, io_dtype);
-    if (need == 0) return GDN_ERR_UNSUPPORTED;
     if (need > (size_t)GDN_STATIC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;   // problem too large
     void* scratch = nullptr;
     const cudaError_t e = scratch_address(&scratch);

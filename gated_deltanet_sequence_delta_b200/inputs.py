@@ -80,14 +80,16 @@ def _rng(seed: int, *stream: int) -> np.random.Generator:
 
 
 _STREAM = {"q": 1, "k": 2, "v": 3, "a": 4, "b": 5, "A_log": 6, "dt": 7, "h0": 8,
-           "lens": 9, "reset": 10, "write": 11}
+           "lens": 9, "reset": 10, "write": 11, "qnorm": 12, "knorm": 13}
 
 _BLOCK = 1 << 24  # elements per generation block, bounds temporary fp32 memory
 
 
-def _normal_rows(rng, rows: int, inner: tuple, dtype: str, unit_norm: bool) -> Tensor:
+def _normal_rows(rng, rows: int, inner: tuple, dtype: str, unit_norm: bool, norm_rng=None,
+                 norm_range=None) -> Tensor:
     """rows x inner standard normals (optionally unit-L2 along the last axis),
-    generated in row blocks and stored in ``dtype``."""
+    generated in row blocks and stored in ``dtype``.  With ``norm_range`` = (lo, hi)
+    each unit row is then given an L2 norm drawn from U(lo, hi) by ``norm_rng``."""
     n_inner = int(np.prod(inner)) if inner else 1
     store_dtype = np.uint16 if dtype == BF16 else np.float32
     out = np.empty((rows,) + tuple(inner), dtype=store_dtype)
@@ -97,6 +99,9 @@ def _normal_rows(rng, rows: int, inner: tuple, dtype: str, unit_norm: bool) -> T
         x = rng.standard_normal((r1 - r0,) + tuple(inner), dtype=np.float32)
         if unit_norm:
             x /= np.sqrt(np.sum(x * x, axis=-1, keepdims=True, dtype=np.float32))
+            if norm_range is not None:
+                lo, hi = norm_range
+                x *= norm_rng.uniform(lo, hi, x.shape[:-1] + (1,)).astype(np.float32)
         out[r0:r1] = f32_to_bf16_bits(x) if dtype == BF16 else x
     return Tensor(out, dtype)
 
@@ -154,11 +159,15 @@ class PrefillInputs:
 def make_prefill(B: int, T: int, HK: int, HV: int, Dk: int, Dv: int, *, io_dtype: str,
                  seed: int, BT: int = 64, h0_std: float = 0.0, cu_seqlens=None,
                  reset_frac: float = 0.0, write_frac: float = 0.0, name: str = "custom",
-                 scale: float = 1.0, l2norm: bool = True) -> PrefillInputs:
-    """Draw one prefill problem with the value recipe in the module docstring."""
+                 scale: float = 1.0, l2norm: bool = True, qk_norm=None) -> PrefillInputs:
+    """Draw one prefill problem with the value recipe in the module docstring.  With
+    ``qk_norm`` = (lo, hi) the q and k rows get L2 norms drawn from U(lo, hi) instead of
+    unit norm (``scale`` and ``l2norm`` are passed to both sides as they are)."""
     rows = B * T
-    q = _normal_rows(_rng(seed, _STREAM["q"]), rows, (HK, Dk), io_dtype, True)
-    k = _normal_rows(_rng(seed, _STREAM["k"]), rows, (HK, Dk), io_dtype, True)
+    q = _normal_rows(_rng(seed, _STREAM["q"]), rows, (HK, Dk), io_dtype, True,
+                     _rng(seed, _STREAM["qnorm"]), qk_norm)
+    k = _normal_rows(_rng(seed, _STREAM["k"]), rows, (HK, Dk), io_dtype, True,
+                     _rng(seed, _STREAM["knorm"]), qk_norm)
     v = _normal_rows(_rng(seed, _STREAM["v"]), rows, (HV, Dv), io_dtype, False)
     a = _rng(seed, _STREAM["a"]).standard_normal((rows, HV), dtype=np.float32)
     b = _rng(seed, _STREAM["b"]).standard_normal((rows, HV), dtype=np.float32)
@@ -269,13 +278,16 @@ class DecodeSetup:
     dt_bias: np.ndarray
     scale: float = 1.0
     l2norm: bool = True
+    qk_norm: tuple | None = None   # (lo, hi): q, k row norms ~ U(lo, hi) instead of 1
 
     def step(self, s: int):
         """Inputs of step ``s``: q, k [B, HK, Dk], v [B, HV, Dv] (Tensor),
         a, b [B, HV] float32.  Each step has its own seeded stream."""
         seed = self.seed
-        q = _normal_rows(_rng(seed, 100, s, 1), self.B, (self.HK, self.Dk), self.io_dtype, True)
-        k = _normal_rows(_rng(seed, 100, s, 2), self.B, (self.HK, self.Dk), self.io_dtype, True)
+        q = _normal_rows(_rng(seed, 100, s, 1), self.B, (self.HK, self.Dk), self.io_dtype, True,
+                         _rng(seed, 100, s, 6), self.qk_norm)
+        k = _normal_rows(_rng(seed, 100, s, 2), self.B, (self.HK, self.Dk), self.io_dtype, True,
+                         _rng(seed, 100, s, 7), self.qk_norm)
         v = _normal_rows(_rng(seed, 100, s, 3), self.B, (self.HV, self.Dv), self.io_dtype, False)
         a = _rng(seed, 100, s, 4).standard_normal((self.B, self.HV), dtype=np.float32)
         b = _rng(seed, 100, s, 5).standard_normal((self.B, self.HV), dtype=np.float32)

@@ -296,8 +296,11 @@ GDN_API gdn_status gdn_chunk_prefill_status(const void* workspace, void* stream,
  *     are rejected with GDN_ERR_WORKSPACE before anything is launched (for bf16, 128-dim
  *     heads that is about 2K tokens at 32 value heads).
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) and caches it; make that first call before any stream
- *     capture on that device.
+ *     (cudaGetSymbolAddress) and caches it.  Under CUDA's lazy module loading (the
+ *     default since CUDA 12.2) that lookup is also what loads the library's device code
+ *     and with it the GDN_STATIC_SCRATCH_BYTES array: a device allocation that can
+ *     synchronise the device.  Make the first call on each device during set-up, before
+ *     the code that must not allocate runs and before any stream capture on that device.
  *   - Every call on a device shares the one array, and it keeps the previous call's
  *     contents; each call rewrites all of it that it reads, so nothing needs clearing.
  *     Calls whose executions overlap on the GPU (other streams, other host threads)
@@ -422,6 +425,28 @@ GDN_API gdn_status gdn_decode_step_fused(const void* x, gdn_dtype io_dtype,
  * NULL argument, CUDA on a CUDA error.
  */
 GDN_API gdn_status gdn_decode_status(int32_t* device_error);
+
+/*
+ * gdn_testing_stall -- a test hook with no counterpart in the method: it lets a test see
+ * a kernel's bounded wait run out without any fault.  With a site other than
+ * GDN_STALL_NONE, later launches of that kernel (from any host thread, on any device)
+ * withhold the copies of one work item of their first CTA, so that the CTA's wait for
+ * them ends at the wait limit (2 s): the kernel records GDN_DEVERR_TIMEOUT, lets what it
+ * did issue land, frees its tensor memory and returns; the outputs of that call are
+ * invalid.  Sites:
+ *   GDN_STALL_DECODE        the staged decode kernel (Dk = Dv = 128: gdn_decode_step,
+ *                           _gated, _fused): the first item's state and rows; reported
+ *                           by gdn_decode_status
+ *   GDN_STALL_PREFILL_PREP  the chunk-local stage of the tensor-core prefill: the first
+ *                           chunk's V tile; reported by gdn_chunk_prefill_status (the
+ *                           state-carry launch of that call then does nothing)
+ * GDN_STALL_NONE restores normal operation.  Not for production use.  Errors: SHAPE for
+ * an unknown site.
+ */
+#define GDN_STALL_NONE 0
+#define GDN_STALL_DECODE 1
+#define GDN_STALL_PREFILL_PREP 2
+GDN_API gdn_status gdn_testing_stall(int32_t site);
 
 #ifdef __cplusplus
 }

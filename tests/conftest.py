@@ -19,3 +19,14 @@ def pytest_configure(config):
 def orc():
     import oracle
     return oracle.default()
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The parity report: one line per comparison the tests made against a reference."""
+    import harness
+    if not harness.PARITY_LOG:
+        return
+    tr = terminalreporter
+    tr.section("parity report: max|err|/RMS(ref), beyond bf16 output rounding, RMS(err)/RMS(ref), bound")
+    for what, mx, arith, rmse, tol in harness.PARITY_LOG:
+        tr.write_line(f"{mx:9.2e} {arith:9.2e} {rmse:9.2e}  <= {tol:g}   {what}")

@@ -36,6 +36,13 @@ def rms_err(got, ref):
 BF16_REP = 2.0 ** -8   # relative representation bound of round-to-nearest bf16
 
 
+# Every comparison made through assert_close, for the run's parity report (printed in the
+# pytest terminal summary): (what, max|err| / RMS(ref), the part of it beyond the output's
+# own bf16 rounding, RMS(err) / RMS(ref), tolerance).  RMS(err) shows a systematic bias that
+# the per-element bound could hide.
+PARITY_LOG: list = []
+
+
 def assert_close(got, ref, tol, what="", out_bf16=False):
     """max|got - ref| <= tol * RMS(ref) (plus 2^-8 |ref| per element when ``got``
     was rounded to bf16).  Returns the arithmetic error relative to RMS(ref)."""
@@ -44,11 +51,14 @@ def assert_close(got, ref, tol, what="", out_bf16=False):
     ref = np.asarray(ref, dtype=np.float64)
     if ref.size == 0:
         return 0.0
-    excess = np.abs(got - ref) - (BF16_REP * np.abs(ref) if out_bf16 else 0.0)
+    d = got - ref
+    excess = np.abs(d) - (BF16_REP * np.abs(ref) if out_bf16 else 0.0)
     arith = float(max(np.max(excess), 0.0))
-    assert arith <= tol * max(rms, 1e-30), (
+    den = max(rms, 1e-30)
+    PARITY_LOG.append((what, err / den, arith / den, float(np.sqrt(np.mean(d * d))) / den, tol))
+    assert arith <= tol * den, (
         f"{what}: max|err| {err:.3e} (beyond output rounding {arith:.3e}) > {tol:g} * RMS {rms:.3e}")
-    return arith / max(rms, 1e-30)
+    return arith / den
 
 
 # ---------------------------------------------------------------------------

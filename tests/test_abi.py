@@ -283,3 +283,27 @@ def test_decode_status_null(L):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(binding.GDNLibraryError):
         binding.lib(str(tmp_path / "nope.so"))
+
+
+def test_static_scratch_entry_point_reports_sizes_like_the_workspace_one(L):
+    """gdn_chunk_prefill_static_ws rejects the sizes gdn_chunk_prefill rejects, with the same
+    status, before it touches its scratch (so no GPU is needed here)."""
+    f = L.gdn_chunk_prefill_static_ws
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    f.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32, i32,
+                  ctypes.c_float, i32, vp, vp, vp]
+    f.restype = ctypes.c_int
+
+    def static(**kw):
+        a = dict(B=1, T=128, N=1, HK=2, HV=4, Dk=128, Dv=128, BT=64, cu=None, io=1)
+        a.update(kw)
+        return f(A, A + 64 * MB, A + 128 * MB, a["io"], A + 192 * MB, A + 200 * MB, None, a["cu"], a["B"], a["T"],
+                 a["N"], a["HK"], a["HV"], a["Dk"], a["Dv"], a["BT"], 1.0, 1, A + 256 * MB, A + 384 * MB, None)
+
+    cases = [dict(HK=2, HV=3), dict(HK=0), dict(B=2, N=1), dict(cu=A + 500 * MB, B=2, N=2), dict(Dk=96),
+             dict(BT=32), dict(T=-1), dict(io=5), dict(cu=A + 500 * MB, T=1 << 31)]
+    for kw in cases:
+        want = _prefill(L, **{k: v for k, v in kw.items() if k != "io"}, **({"io": kw["io"]} if "io" in kw else {}))
+        assert want != 0, kw
+        assert static(**kw) == want, (kw, static(**kw), want)
+    assert static(HK=2, HV=3) == 2   # GDN_ERR_SHAPE, as gdn_chunk_prefill

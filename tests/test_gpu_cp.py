@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 from gated_deltanet_sequence_delta_b200 import inputs as I
-from harness import TOL, assert_close, gpu_gates, to_dev, to_np
+from harness import TOL, assert_close, gpu_gates, oracle_gates, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -37,9 +37,10 @@ def _run(io, R, T_seg, N, HK, HV, seed):
         finals.append(final)
         starts.append(start)
     o_cp = torch.cat(outs, dim=1)
-    # oracle over the whole sequences, on the same rounded inputs and the GPU's gates
+    # oracle over the whole sequences, on the same rounded inputs, with its own gates
+    g_ref, b_ref = oracle_gates(inp)
     o_ref, h_ref = oracle.recurrence(inp.q.f64().reshape(N, T, HK, 128), inp.k.f64().reshape(N, T, HK, 128),
-                                     inp.v.f64().reshape(N, T, HV, 128), to_np(g), to_np(beta),
+                                     inp.v.f64().reshape(N, T, HV, 128), g_ref, b_ref,
                                      h0=inp.h0.astype(np.float64))
     tol = TOL[io]
     assert_close(to_np(o_cp), o_ref, tol, f"context-parallel o ({io})", out_bf16=io == I.BF16)
@@ -48,8 +49,8 @@ def _run(io, R, T_seg, N, HK, HV, seed):
     # every rank's start state is the state at its segment's first token
     _, h_mid = oracle.recurrence(inp.q.f64().reshape(N, T, HK, 128)[:, :T_seg * 2],
                                  inp.k.f64().reshape(N, T, HK, 128)[:, :T_seg * 2],
-                                 inp.v.f64().reshape(N, T, HV, 128)[:, :T_seg * 2], to_np(g)[:, :T_seg * 2],
-                                 to_np(beta)[:, :T_seg * 2], h0=inp.h0.astype(np.float64))
+                                 inp.v.f64().reshape(N, T, HV, 128)[:, :T_seg * 2], g_ref[:, :T_seg * 2],
+                                 b_ref[:, :T_seg * 2], h0=inp.h0.astype(np.float64))
     assert_close(to_np(starts[2]), h_mid, tol, "start state of segment 2")
     assert G.gdn_cp_status() == 0
 
@@ -82,3 +83,34 @@ def test_cp_segment_matches_two_prefills():
     assert torch.equal(o, o2) and torch.equal(hT, hT2)
     assert_close(to_np(c), to_np(c2), TOL[I.BF16], "c", out_bf16=True)
     assert_close(to_np(A), to_np(A2), TOL[I.BF16], "A")
+
+
+def test_cp_product_function_through_a_process_group():
+    """context_parallel.cp_chunk_prefill as a user calls it: a real NCCL process group of
+    one rank on this GPU, so that gather_transitions runs its all-gathers on CUDA tensors
+    and gdn_cp_combine consumes what they return; against the oracle."""
+    import datetime
+    import oracle
+    import torch
+    import torch.distributed as dist
+    from gated_deltanet_sequence_delta_b200 import context_parallel as CP
+    N, T, HK, HV = 2, 300, 2, 4
+    inp = I.make_prefill(N, T, HK, HV, 128, 128, io_dtype=I.BF16, seed=94, h0_std=0.02)
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        g, beta = gpu_gates(inp)
+        o, final, start = CP.cp_chunk_prefill(to_dev(inp.q), to_dev(inp.k), to_dev(inp.v), g.view(N, T, HV),
+                                              beta.view(N, T, HV), initial_state=to_dev(inp.h0))
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    g_ref, b_ref = oracle_gates(inp)
+    o_ref, h_ref = oracle.recurrence(inp.q.f64(), inp.k.f64(), inp.v.f64(), g_ref, b_ref,
+                                     h0=inp.h0.astype(np.float64))
+    tol = TOL[I.BF16]
+    assert_close(to_np(o), o_ref, tol, "cp_chunk_prefill, one rank: o", out_bf16=True)
+    assert_close(to_np(final), h_ref, tol, "cp_chunk_prefill, one rank: final state")
+    # the only segment starts from the initial state
+    assert_close(to_np(start), inp.h0.astype(np.float64), 1e-6, "cp_chunk_prefill, one rank: start state")
