@@ -109,12 +109,10 @@ __device__ __forceinline__ bool locate_chunk(int chunk, const int32_t* __restric
 // ======================================================================================
 __global__ void __launch_bounds__(1024) chunk_table_kernel(const int32_t* __restrict__ cu, int n_seqs,
                                                            int64_t T, int32_t* __restrict__ chunk_off,
-                                                           int32_t* __restrict__ status,
-                                                           int32_t* __restrict__ flags, int64_t n_flags) {
+                                                           int32_t* __restrict__ status) {
     __shared__ int s_part[1024];
     __shared__ int s_bad;
     const int tid = threadIdx.x;
-    for (int64_t i = tid; i < n_flags; i += 1024) flags[i] = 0;   // ready flags of the fused launch
     if (tid == 0) s_bad = 0;
     __syncthreads();
     const int per = (n_seqs + 1023) / 1024;
@@ -198,7 +196,7 @@ __device__ __forceinline__ void frag_b(uint32_t* b, const float (*M)[65], int r0
 
 // Block row I of T: warp j (< I) forms X_j = sum_{k=j}^{I-1} L_Ik T_kj, then T_Ij = -T_II X_j.
 template <int I>
-__device__ __forceinline__ void tinv_row_block(float (*M)[65], float (*X)[16][17], int tid, int bar) {
+__device__ __forceinline__ void tinv_row_block(float (*M)[65], float (*X)[16][17], int tid) {
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
     const float(*Xc)[17] = nullptr;
     if (warp < I) {
@@ -224,7 +222,7 @@ __device__ __forceinline__ void tinv_row_block(float (*M)[65], float (*X)[16][17
             X[j][g + 8][8 * nt + 2 * q + 1] = acc[nt][3];
         }
     }
-    tc::named_bar(bar, 128);   // every read of row block I of L is done before it is overwritten
+    __syncthreads();   // every read of row block I of L is done before it is overwritten
     if (warp < I) {
         const int j = warp;
         Xc = X[j];
@@ -245,12 +243,10 @@ __device__ __forceinline__ void tinv_row_block(float (*M)[65], float (*X)[16][17
             M[16 * I + g + 8][16 * j + 8 * nt + 2 * q + 1] = -acc[nt][3];
         }
     }
-    tc::named_bar(bar, 128);
+    __syncthreads();
 }
 
-// The 128 threads of one worker run it; `bar` is their named barrier (0 when they are the
-// whole CTA).
-__device__ __forceinline__ void tinv64_inplace(float (*M)[65], float (*X)[16][17], int tid, int bar) {
+__device__ __forceinline__ void tinv64_inplace(float (*M)[65], float (*X)[16][17], int tid) {
     float col[16];
     const int b = tid >> 4, c = tid & 15, o = 16 * b;
     if (tid < 64) {
@@ -263,16 +259,16 @@ __device__ __forceinline__ void tinv64_inplace(float (*M)[65], float (*X)[16][17
             for (int i = j + 1; i < 16; ++i) col[i] = fmaf(-M[o + i][o + j], xj, col[i]);
         }
     }
-    tc::named_bar(bar, 128);   // all reads of the diagonal blocks of L precede their overwrite
+    __syncthreads();   // all reads of the diagonal blocks of L precede their overwrite
     if (tid < 64) {
 #pragma unroll
         for (int i = 1; i < 16; ++i)
             if (i > c) M[o + i][o + c] = col[i];
     }
-    tc::named_bar(bar, 128);
-    tinv_row_block<1>(M, X, tid, bar);
-    tinv_row_block<2>(M, X, tid, bar);
-    tinv_row_block<3>(M, X, tid, bar);
+    __syncthreads();
+    tinv_row_block<1>(M, X, tid);
+    tinv_row_block<2>(M, X, tid);
+    tinv_row_block<3>(M, X, tid);
 }
 
 // ======================================================================================
@@ -289,7 +285,6 @@ struct PrepSmem {
     float X[3][16][17];
     float rk[64], rq[64], G[64], bt[64], bgr[64], red[8];
     float eu[64];   // rk_j exp(G_r - G_j), the token factor of the separated decays
-    float dd[64];   // exp(G_C - G_j): the decay from token j to the chunk's end (K_tilde rows)
     float ga[2][64], ba[2][64];   // g, beta of value head gi in slot gi % 2, loaded ahead
     uint64_t bar_load, bar_v, bar_mma;
     uint32_t tmem_base;
@@ -320,72 +315,37 @@ __device__ __forceinline__ void store_tile_from_tmem(f16* __restrict__ dst, uint
     }
 }
 
-// Row t = tid of a 128 x 64 fp16 tile from TMEM lane t (64 fp32 columns), stored as one
-// contiguous 128-byte row: the tile's transpose in the layout the MMA produced it.
-__device__ __forceinline__ void store_rows_from_tmem(f16* __restrict__ dst, uint32_t taddr, int tid) {
-    uint4* d = reinterpret_cast<uint4*>(dst + (size_t)tid * 64);
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {
-        float w[32];
-        tc::tmem_ld32(taddr + part * 32, w);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint4 u;
-            u.x = pack_h2(w[8 * c + 0], w[8 * c + 1]);
-            u.y = pack_h2(w[8 * c + 2], w[8 * c + 3]);
-            u.z = pack_h2(w[8 * c + 4], w[8 * c + 5]);
-            u.w = pack_h2(w[8 * c + 6], w[8 * c + 7]);
-            d[part * 4 + c] = u;
-        }
+template <int G>
+__global__ void __launch_bounds__(128, 4)
+chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                  const float* __restrict__ beta, const int32_t* __restrict__ cu,
+                  const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HV, float scale,
+                  int l2norm, int HK, f16* __restrict__ Wg, f16* __restrict__ Ug, f16* __restrict__ Pg,
+                  f16* __restrict__ QKg, float* __restrict__ SCg, int32_t* __restrict__ status, int stall) {
+    extern __shared__ uint8_t smem_raw[];
+    PrepSmem& S = *reinterpret_cast<PrepSmem*>(align1024(smem_raw));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int chunk = blockIdx.x, hk = blockIdx.y;
+    if (*reinterpret_cast<volatile int32_t*>(status) != 0) return;
+    int n, cn;
+    int64_t s;
+    if (!locate_chunk(chunk, chunk_off, cu, T, n_seqs, n, s, cn)) return;
+
+    if (warp == 0) {
+        tc::tmem_alloc(&S.tmem_base, kPrepTmemCols);
+        tc::tmem_relinquish();
     }
-}
-
-// Where one worker's chunk-local results go.
-struct PrepOut {
-    f16* W;          // [rows, 128]: W of each (chunk, value head), 64 rows
-    f16* U;          // two-kernel path: [rows, 128] U * 2^-e (e per chunk and value head); fused: its
-                     //   transpose, [(chunk, value head) * 128 + value, 64 tokens]
-    f16* P;          // [rows, 64]: P (two-kernel path) or P^T (fused path)
-    f16* QK;         // two-kernel path: [K_hat; Q_hat] per (chunk, q/k head), 128 rows; fused: Q_hat, 64 rows
-    float* SC;       // [chunks * HV, SC_FLOATS] per-row scalars
-    f16* Kt;         // fused: K_tilde = diag(exp(G_C - G)) K_hat per (chunk, value head), 64 rows
-    int32_t* flags;  // fused: per (chunk, q/k head) ready flag, set once all of the above are written
-};
-
-// Barrier phases a worker carries from one item to the next.
-struct PrepPhases {
-    uint32_t load = 0;     // parity of the next K / Q tile wait
-    uint32_t mma = 0;      // parity of the next product wait
-    uint32_t vcount = 0;   // V tile copies issued so far
-};
-
-// The chunk-local stage for one (chunk, q/k head) item, run by 128 threads (tid 0-127, their
-// TMEM lanes 0-127 at column base `tmem`, named barrier `bar`).  Returns false if a bounded
-// wait gave up (recorded in `status`; what was issued has landed again on return).
-// FUSED writes P^T, Q_hat alone and K_tilde per value head (the operands of the fused
-// carry), then raises the item's ready flag.
-// issue the K and Q tile copies of item (chunk at token s, q/k head hk) on bar_load (one thread)
-__device__ __forceinline__ void prep_load_kq(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMap* tm_k, int hk,
-                                             int si) {
-    uint8_t* kq = reinterpret_cast<uint8_t*>(&S.KQ[0][0]);
-    tc::mbar_expect_tx(&S.bar_load, 4 * 64 * 64 * 2);
-    tc::tma_load_3d(kq, tm_k, &S.bar_load, 0, hk, si);
-    tc::tma_load_3d(kq + 16384, tm_k, &S.bar_load, 64, hk, si);
-    tc::tma_load_3d(kq + 8192, tm_q, &S.bar_load, 0, hk, si);
-    tc::tma_load_3d(kq + 16384 + 8192, tm_q, &S.bar_load, 64, hk, si);
-}
-
-// FUSED: `loaded` says this item's K, Q copies were issued by the item before; next_hk >= 0 asks
-// for the next item's copies (q/k head next_hk at token next_s) to be issued at the end, before
-// the release of this item's flag, so that their latency overlaps it.
-template <int G, bool FUSED>
-__device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                          const float* __restrict__ g, const float* __restrict__ beta, int chunk, int hk, int64_t s,
-                          int cn, int HV, int HK, float scale, int l2norm, const PrepOut& out,
-                          int32_t* __restrict__ status, bool stall, uint32_t tmem, int tid, int bar, PrepPhases& ph,
-                          bool loaded = false, int next_hk = -1, int64_t next_s = 0) {
-    const int warp = tid >> 5;
+    if (tid == 32) {
+        tc::mbar_init(&S.bar_load, 1);
+        tc::mbar_init(&S.bar_v, 1);
+        tc::mbar_init(&S.bar_mma, 1);
+        tc::fence_mbar_init();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     // TMEM: columns 0-63 the Gram tiles (kept for every value head), 64-127 W^T; U^T goes
     // to 64-127 after W^T is read out, except for the last value head, whose U^T takes the
@@ -393,12 +353,16 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
     const uint32_t tG = tmem, tW = tmem + 64;
     const int si = (int)s;
     uint8_t* kq = reinterpret_cast<uint8_t*>(&S.KQ[0][0]);
-    const uint32_t load_par = ph.load;
-    ph.load ^= 1u;
-    const uint32_t vbase = ph.vcount;   // V copies of earlier items
-    bool ok;
+    uint32_t mma_phase = 0;
+    int v_loads = 0;   // V tile copies issued (thread 0)
 
-    if (tid == 0 && !loaded) prep_load_kq(S, tm_q, tm_k, hk, si);
+    if (tid == 0) {
+        tc::mbar_expect_tx(&S.bar_load, 4 * 64 * 64 * 2);
+        tc::tma_load_3d(kq, &tm_k, &S.bar_load, 0, hk, si);
+        tc::tma_load_3d(kq + 16384, &tm_k, &S.bar_load, 64, hk, si);
+        tc::tma_load_3d(kq + 8192, &tm_q, &S.bar_load, 0, hk, si);
+        tc::tma_load_3d(kq + 16384 + 8192, &tm_q, &S.bar_load, 64, hk, si);
+    }
     if (tid < 64) {   // gates of the group's first two value heads, under the TMA latency
 #pragma unroll
         for (int gi = 0; gi < (G < 2 ? G : 2); ++gi) {
@@ -407,8 +371,8 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
             S.ba[gi][tid] = tid < cn ? beta[(s + tid) * HV + h] : 0.f;
         }
     }
-    ok = tc::mbar_wait(&S.bar_load, load_par);
-    if (tc::named_bar_any(bar, 128, !ok)) goto abort;
+    bool ok = tc::mbar_wait(&S.bar_load, 0);
+    if (__syncthreads_or(!ok)) goto abort;
 
     // ---- Gram tiles: D_G[0:64] = K K^T, D_G[64:128] = Q K^T (bf16, M=128, N=64, K=Dk) ----
     if (tid == 0) {
@@ -441,9 +405,9 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
         if (tid < 64) S.rk[tid] = l2_inv(ss, l2norm);
         else S.rq[tid - 64] = l2_inv(ss, l2norm);
     }
-    ok = tc::mbar_wait(&S.bar_mma, ph.mma);
-    ph.mma ^= 1u;
-    if (tc::named_bar_any(bar, 128, !ok)) goto abort;
+    ok = tc::mbar_wait(&S.bar_mma, mma_phase);
+    mma_phase ^= 1;
+    if (__syncthreads_or(!ok)) goto abort;
     tc::tc_fence_after();
     {
         const float rki = tid < 64 ? S.rk[tid] : 0.f;
@@ -451,9 +415,7 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
         {   // K_hat (tid < 64) / Q_hat row: fp16 in place (K_hat feeds the W MMA) and out to
             // global in natural column order; rows past the chunk are zeroed
             const float rr = tid < cn || (tid >= 64 && tid - 64 < cn) ? (tid < 64 ? rki : rqi) : 0.f;
-            uint4* dst = nullptr;
-            if (!FUSED) dst = reinterpret_cast<uint4*>(out.QK + (((size_t)chunk * HK + hk) * 128 + tid) * D);
-            else if (tid >= 64) dst = reinterpret_cast<uint4*>(out.QK + (((size_t)chunk * HK + hk) * 64 + tid - 64) * D);
+            uint4* dst = reinterpret_cast<uint4*>(QKg + (((size_t)chunk * HK + hk) * 128 + tid) * D);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint4* row = reinterpret_cast<uint4*>(kq + half * 16384 + tid * 128);
@@ -467,21 +429,19 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
                     for (int t = 0; t < 8; ++t) hx[t] = __float2half_rn(__bfloat162float(e[t]) * rr);
                     const uint4 hv = *reinterpret_cast<const uint4*>(hx);
                     row[pc] = hv;
-                    if (dst) dst[half * 8 + c16] = hv;
+                    dst[half * 8 + c16] = hv;
                 }
             }
         }
         tc::fence_async_smem();
-        tc::named_bar(bar, 128);
+        __syncthreads();
         // Q is consumed: its rows now receive V of the first value head (test hook,
-        // gdn_testing_stall: not for the first item, whose wait for it then runs out)
-        if (!FUSED && !stall) {
-            ++ph.vcount;   // every thread counts the copies: the parity of each V wait follows from it
-            if (tid == 0) {
-                tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
-                tc::tma_load_3d(kq + 8192, tm_v, &S.bar_v, 0, hk * G, si);
-                tc::tma_load_3d(kq + 16384 + 8192, tm_v, &S.bar_v, 64, hk * G, si);
-            }
+        // gdn_testing_stall: not for the first CTA, whose wait for it then runs out)
+        if (tid == 0 && !(stall && chunk == 0 && hk == 0)) {
+            tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+            ++v_loads;
+            tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, hk * G, si);
+            tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, hk * G, si);
         }
 
         for (int gi = 0; gi < G; ++gi) {
@@ -499,13 +459,13 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
                 S.G[tid] = gv;
                 S.bt[tid] = S.ba[gi & 1][tid];
             }
-            tc::named_bar(bar, 128);
+            __syncthreads();
             if (G > 2 && gi + 2 < G && tid < 64) {   // slot gi % 2 is read: value head gi + 2's gates
                 S.ga[gi & 1][tid] = tid < cn ? g[(s + tid) * HV + h + 2] : 0.f;
                 S.ba[gi & 1][tid] = tid < cn ? beta[(s + tid) * HV + h + 2] : 0.f;
             }
             if (tid >= 32 && tid < 64) S.G[tid] += S.G[31];
-            tc::named_bar(bar, 128);
+            __syncthreads();
             if (tid < 64) S.bgr[tid] = S.bt[tid] * expf(S.G[tid]);
             const float Gl = S.G[63];   // padding adds 0, so this is G at the last token
             // exp(G_i - G_j) = exp(G_i - G_r) exp(G_r - G_j) with G_r = G_last / 2: both
@@ -515,7 +475,7 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
             const float Gr = 0.5f * Gl;
             if (sep) {
                 if (tid < 64) S.eu[tid] = S.rk[tid] * __expf(Gr - S.G[tid]);
-                tc::named_bar(bar, 128);
+                __syncthreads();
             }
             // ---- L (strictly lower) into M, P (lower incl. diagonal) out, scalars; the
             //      Gram row of this thread is read back from TMEM --------------------------
@@ -539,80 +499,31 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
                             S.M[i][j] = v;
                         }
                     }
-                    const float di = i < cn ? expf(Gl - Gi) : 0.f;
-                    out.SC[ch * SC_FLOATS + 64 + i] = di;
-                    if (FUSED) S.dd[i] = di;
+                    SCg[ch * SC_FLOATS + 64 + i] = i < cn ? expf(Gl - Gi) : 0.f;
                 } else {
                     const int i = tid - 64;
                     const float Gi = S.G[i], qi = scale * rqi;
-                    out.SC[ch * SC_FLOATS + i] = i < cn ? scale * expf(Gi) : 0.f;
-                    if (i == 0) out.SC[ch * SC_FLOATS + SC_GC] = expf(Gl);
+                    SCg[ch * SC_FLOATS + i] = i < cn ? scale * expf(Gi) : 0.f;
+                    if (i == 0) SCg[ch * SC_FLOATS + SC_GC] = expf(Gl);
+                    uint4* prow = reinterpret_cast<uint4*>(Pg + (ch * 64 + i) * 64);
                     const float ai = sep && i < cn ? qi * __expf(Gi - Gr) : 0.f;
-                    if (!FUSED) {
-                        uint4* prow = reinterpret_cast<uint4*>(out.P + (ch * 64 + i) * 64);
 #pragma unroll
-                        for (int c8 = 0; c8 < 8; ++c8) {
-                            __align__(16) f16 e[8];
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        __align__(16) f16 e[8];
 #pragma unroll
-                            for (int t = 0; t < 8; ++t) {
-                                const int j = c8 * 8 + t;
-                                float v = 0.f;
-                                if (sep) v = j <= i ? ai * S.eu[j] * row[j] : 0.f;
-                                else if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
-                                e[t] = __float2half_rn(v);
-                            }
-                            prow[c8] = *reinterpret_cast<const uint4*>(e);
-                        }
-                    } else {   // P^T: P[i][j] at row j, column i of a staging tile (the V rows of K / Q
-                               // half 0, free until this head's V is loaded); a warp writes 64
-                               // contiguous bytes per j
-                        f16* pst = reinterpret_cast<f16*>(kq + 8192) + i;
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) {
+                        for (int t = 0; t < 8; ++t) {
+                            const int j = c8 * 8 + t;
                             float v = 0.f;
                             if (sep) v = j <= i ? ai * S.eu[j] * row[j] : 0.f;
                             else if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
-                            pst[j * 64] = __float2half_rn(v);
+                            e[t] = __float2half_rn(v);
                         }
+                        prow[c8] = *reinterpret_cast<const uint4*>(e);
                     }
                 }
             }
-            tc::named_bar(bar, 128);
-            if (FUSED) {
-                // K_tilde = diag(d) K_hat and P^T out, 16 bytes per thread and copy, 16 consecutive
-                // threads on one row: every store instruction covers whole rows
-#pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    const int m = tid + 128 * r, krow = m >> 4, c16 = m & 15;
-                    const uint4 u = *reinterpret_cast<const uint4*>(kq + (c16 >> 3) * 16384 + krow * 128 +
-                                                                    (((c16 & 7) ^ (krow & 7)) << 4));
-                    const __half2* e = reinterpret_cast<const __half2*>(&u);
-                    const __half2 dd = __float2half2_rn(S.dd[krow]);
-                    uint4 o4;
-                    __half2* oh = reinterpret_cast<__half2*>(&o4);
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) oh[t] = __hmul2(e[t], dd);
-                    reinterpret_cast<uint4*>(out.Kt + (ch * 64 + krow) * D)[c16] = o4;
-                }
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int m = tid + 128 * r;   // 16-byte piece m of the 8 KB P^T tile
-                    reinterpret_cast<uint4*>(out.P + ch * 64 * 64)[m] = reinterpret_cast<const uint4*>(kq + 8192)[m];
-                }
-                // the staging tile is read: this head's V may now overwrite it (the copies run
-                // under the inverse below)
-                tc::fence_async_smem();
-                tc::named_bar(bar, 128);
-                if (!(stall && gi == 0)) {
-                    ++ph.vcount;
-                    if (tid == 0) {
-                        tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
-                        tc::tma_load_3d(kq + 8192, tm_v, &S.bar_v, 0, h, si);
-                        tc::tma_load_3d(kq + 16384 + 8192, tm_v, &S.bar_v, 64, h, si);
-                    }
-                }
-            }
-            tinv64_inplace(S.M, S.X, tid, bar);
+            __syncthreads();
+            tinv64_inplace(S.M, S.X, tid);
             // ---- fp16 MMA operands T diag(b gamma) and T diag(b), 128B-swizzled, written
             //      over M once every thread holds its part of T -----------------------------
             {
@@ -623,7 +534,7 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
                     const int j = c0 + t;
                     tv[t] = j < i ? S.M[i][j] : (j == i ? 1.f : 0.f);
                 }
-                tc::named_bar(bar, 128);
+                __syncthreads();
                 uint8_t* aw = reinterpret_cast<uint8_t*>(&S.M[0][0]);
                 uint8_t* au = aw + 8192;
 #pragma unroll
@@ -642,8 +553,8 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
             }
             // ---- V tile of this head: max |v|, then fp16(v * sv) in place, rows past the
             //      chunk zeroed -----------------------------------------------------------
-            ok = tc::mbar_wait(&S.bar_v, (vbase + (uint32_t)gi) & 1u);
-            if (tc::named_bar_any(bar, 128, !ok)) goto abort;
+            ok = tc::mbar_wait(&S.bar_v, gi & 1);
+            if (__syncthreads_or(!ok)) goto abort;
             {
                 const int r = tid >> 1, half = tid & 1;
                 uint4* vr = reinterpret_cast<uint4*>(kq + half * 16384 + 8192 + r * 128);
@@ -660,7 +571,7 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
                 if ((tid & 31) == 0) S.red[warp] = vmax;
-                tc::named_bar(bar, 128);
+                __syncthreads();
                 vmax = fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3]));
                 const float uinv = pow2_above(vmax), sv = r < cn ? 1.f / uinv : 0.f;
 #pragma unroll
@@ -674,13 +585,13 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
                     vr[pc] = *reinterpret_cast<const uint4*>(hx);
                 }
                 if (tid == 0) {
-                    out.SC[ch * SC_FLOATS + SC_UINV] = uinv;
-                    out.SC[ch * SC_FLOATS + SC_VMAX] = vmax;
+                    SCg[ch * SC_FLOATS + SC_UINV] = uinv;
+                    SCg[ch * SC_FLOATS + SC_VMAX] = vmax;
                 }
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
-            tc::named_bar(bar, 128);
+            __syncthreads();
             // ---- W^T = K_hat^T AW^T and (V sv)^T AU^T (fp16, M=128, N=64, K=64 tokens) ----
             const uint32_t kb = tc::smem_u32(kq), vb = kb + 8192;
             const uint32_t awb = tc::smem_u32(&S.M[0][0]), aub = awb + 8192;
@@ -699,15 +610,15 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
                 }
                 tc::mma_commit(&S.bar_mma);
             }
-            ok = tc::mbar_wait(&S.bar_mma, ph.mma);
-            ph.mma ^= 1u;
-            if (tc::named_bar_any(bar, 128, !ok)) goto abort;
+            ok = tc::mbar_wait(&S.bar_mma, mma_phase);
+            mma_phase ^= 1;
+            if (__syncthreads_or(!ok)) goto abort;
             tc::tc_fence_after();
             // ---- epilogue: lane t of D_W / D_U is column t of W / U -----------------------
-            store_tile_from_tmem(out.W + ch * 64 * D, tW + lane_base, tid);
+            store_tile_from_tmem(Wg + ch * 64 * D, tW + lane_base, tid);
             if (!last) {   // U^T into the W^T columns once they are read
                 tc::tc_fence_before();
-                tc::named_bar(bar, 128);
+                __syncthreads();
                 if (tid == 0) {
                     tc::tc_fence_after();
 #pragma unroll
@@ -716,89 +627,37 @@ __device__ bool prep_item(PrepSmem& S, const CUtensorMap* tm_q, const CUtensorMa
                                      tc::desc_sw128(aub + kk * 32, 16, 1024), idx, kk > 0);
                     tc::mma_commit(&S.bar_mma);
                 }
-                ok = tc::mbar_wait(&S.bar_mma, ph.mma);
-                ph.mma ^= 1u;
-                if (tc::named_bar_any(bar, 128, !ok)) goto abort;
+                ok = tc::mbar_wait(&S.bar_mma, mma_phase);
+                mma_phase ^= 1;
+                if (__syncthreads_or(!ok)) goto abort;
                 tc::tc_fence_after();
-                if (!FUSED) {
-                    ++ph.vcount;
-                    if (tid == 0) {   // the V rows are free again: next head's V
-                        tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
-                        tc::tma_load_3d(kq + 8192, tm_v, &S.bar_v, 0, h + 1, si);
-                        tc::tma_load_3d(kq + 16384 + 8192, tm_v, &S.bar_v, 64, h + 1, si);
-                    }
+                if (tid == 0) {   // the V rows are free again: next head's V
+                    tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+                    ++v_loads;
+                    tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, h + 1, si);
+                    tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, h + 1, si);
                 }
             }
-            if (FUSED) store_rows_from_tmem(out.U + ch * 128 * 64, (last ? tG : tW) + lane_base, tid);
-            else store_tile_from_tmem(out.U + ch * 64 * D, (last ? tG : tW) + lane_base, tid);
+            store_tile_from_tmem(Ug + ch * 64 * D, (last ? tG : tW) + lane_base, tid);
             tc::tc_fence_before();
-            tc::named_bar(bar, 128);   // TMEM reads done; M (the operands) free for the next head
+            __syncthreads();   // TMEM reads done; M (the operands) free for the next head
         }
     }
-    // the next item's tile copies overwrite what this one wrote to the tiles with generic stores
-    tc::fence_async_smem();
     tc::tc_fence_before();
-    tc::named_bar(bar, 128);
-    if (FUSED) {
-        if (tid == 0 && next_hk >= 0) prep_load_kq(S, tm_q, tm_k, next_hk, (int)next_s);
-        // every thread's writes of this item, then the flag (release, GPU scope)
-        __threadfence();
-        tc::named_bar(bar, 128);
-        if (tid == 0) {
-            asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(out.flags + (size_t)chunk * HK + hk), "r"(1)
-                         : "memory");
-        }
-    }
-    return true;
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kPrepTmemCols);
+    return;
 abort:
     if (tid == 0) {
         record_timeout(status);
         // the copies and products still in flight land before the shared memory and TMEM are
-        // released or reused; each wait is for the latest phase of its barrier (at once if
-        // complete)
-        (void)tc::mbar_wait(&S.bar_load, load_par, 50000000ull);
-        if (ph.vcount > vbase) (void)tc::mbar_wait(&S.bar_v, (ph.vcount - 1u) & 1u, 50000000ull);
-        (void)tc::mbar_wait(&S.bar_mma, ph.mma ^ 1u, 50000000ull);
-    }
-    tc::tc_fence_before();
-    tc::named_bar(bar, 128);
-    return false;
-}
-
-// The chunk-local stage of the two-kernel path: one CTA per (chunk, q/k head), four per SM.
-template <int G>
-__global__ void __launch_bounds__(128, 4)
-chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
-                  const float* __restrict__ beta, const int32_t* __restrict__ cu,
-                  const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HV, float scale,
-                  int l2norm, int HK, PrepOut out, int32_t* __restrict__ status, int stall) {
-    extern __shared__ uint8_t smem_raw[];
-    PrepSmem& S = *reinterpret_cast<PrepSmem*>(align1024(smem_raw));
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int chunk = blockIdx.x, hk = blockIdx.y;
-    if (*reinterpret_cast<volatile int32_t*>(status) != 0) return;
-    int n, cn;
-    int64_t s;
-    if (!locate_chunk(chunk, chunk_off, cu, T, n_seqs, n, s, cn)) return;
-
-    if (warp == 0) {
-        tc::tmem_alloc(&S.tmem_base, kPrepTmemCols);
-        tc::tmem_relinquish();
-    }
-    if (tid == 32) {
-        tc::mbar_init(&S.bar_load, 1);
-        tc::mbar_init(&S.bar_v, 1);
-        tc::mbar_init(&S.bar_mma, 1);
-        tc::fence_mbar_init();
+        // released; each wait is for the latest phase of its barrier (at once if complete)
+        (void)tc::mbar_wait(&S.bar_load, 0, 50000000ull);
+        if (v_loads > 0) (void)tc::mbar_wait(&S.bar_v, (uint32_t)((v_loads - 1) & 1), 50000000ull);
+        (void)tc::mbar_wait(&S.bar_mma, mma_phase ^ 1u, 50000000ull);
     }
     tc::tc_fence_before();
     __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = S.tmem_base;
-    PrepPhases ph;
-    (void)prep_item<G, false>(S, &tm_q, &tm_k, &tm_v, g, beta, chunk, hk, s, cn, HV, HK, scale, l2norm, out, status,
-                              stall && chunk == 0 && hk == 0, tmem, tid, 0, ph);
     if (warp == 0) tc::tmem_dealloc(tmem, kPrepTmemCols);
 }
 // ======================================================================================
@@ -1285,518 +1144,6 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
 }
 
 // ======================================================================================
-// Fused prefill: one cooperative launch, one CTA per SM.  CTAs [0, n_carry) carry the state
-// of the (sequence, value head) chains; the others each hold four chunk-local workers
-// (prep_item, FUSED) that run through the (chunk, q/k head) items in chunk order and raise a
-// ready flag per item.  The carry waits on those flags, so the chunk-local work of later
-// chunks runs while the state is carried through earlier ones; no worker ever waits on the
-// carry, so neither side can block the other.
-//
-// Carry CTA, per chain (sequence n, value head h) and chunk (64 tokens), with the state
-// held transposed in TMEM (lane v = value column v, H^T[v][k] = H[k][v]):
-//   D1 = H^T [W; Q_hat]^T          A = H^T (fp16, TMEM), B = [W; Q_hat] (K-major)   8 MMAs, N = 128
-//        -> columns 0-63: (W H)^T, columns 64-127: (Q_hat H)^T
-//   Delta^T = U^T - (W H)^T        (epilogue, into TMEM as the next A operand)
-//   D2 += Delta^T [K_tilde | P^T]  A = Delta^T (TMEM),  B MN-major                   4 MMAs, N = 192
-//        -> columns 0-127 accumulate onto gamma_C H^T: the new state H^T (fp32, never leaves
-//           TMEM but for its fp16 operand copy); columns 128-191: (P Delta)^T
-//   O = diag(a) Q_hat H + P Delta  (output warps)
-// so 12 tensor-core instructions per chunk and head (the instruction count, not the FLOPs,
-// sets a tensor-core step's time).  The fp16 operands carry a data scale sc = 2^-e chosen per
-// chunk from the exact max |H| of the state and max |v| of the chunk, so a quiet stretch that
-// follows a loud one keeps its precision.
-// Warps: 0 producer (flags, TMA), 1 MMA issue, 4-11 state epilogue (lane group w % 4, value
-// column v; half (w - 4) / 4 of the K or token columns), 12-15 outputs.
-// ======================================================================================
-constexpr int kFcThreads = 512;
-struct FcStage {
-    uint8_t B1[2][128 * 128];   // [W; Q_hat]: rows 0-63 W, 64-127 Q_hat; K-major 128B-swizzled K halves
-    uint8_t B2[3][64 * 128];    // K_tilde (two 64-column halves) and P^T: MN-major 128B-swizzled
-    uint8_t U[128 * 128];       // U^T * 2^-e: [128 values][64 tokens], 128B-swizzled rows
-    float SC[SC_FLOATS];
-};
-struct FcSmem {
-    FcStage st[2];
-    float red[2][8];            // max |H| per epilogue warp, alternating buffers
-    float scale[4];             // data scale sc of step it, at it % 4
-    float nxt[4][2];            // gamma_C and max |v| of step it, at it % 4, ahead of its stage
-    uint64_t full[2], empty[2], d1, d2, h_ready, d_ready, ofree1, ofree2, scal[4];
-    volatile int abort;
-    int issued;                 // steps whose copies the producer has started
-};
-constexpr uint32_t kFcTx = (uint32_t)sizeof(FcStage);
-static_assert(sizeof(FcStage) % 1024 == 0 && offsetof(FcStage, B2) % 1024 == 0 && offsetof(FcStage, U) % 1024 == 0 &&
-                  offsetof(FcStage, SC) % 16 == 0,
-              "fused carry stage layout");
-constexpr size_t kPrepSlot = (sizeof(PrepSmem) + 1023) / 1024 * 1024;
-constexpr size_t kFusedSmemBytes = (4 * kPrepSlot > sizeof(FcSmem) ? 4 * kPrepSlot : sizeof(FcSmem)) + 1024;
-static_assert(kFusedSmemBytes <= 227 * 1024, "fused prefill: shared memory over the per-block limit");
-// TMEM columns of a carry CTA
-constexpr uint32_t kFcD1 = 0, kFcD2 = 128, kFcA1 = 320, kFcA2 = 384;
-
-struct FusedArgs {
-    const float* g;
-    const float* beta;
-    const int32_t* cu;
-    const int32_t* chunk_off;
-    int64_t T;
-    int n_seqs, HK, HV;
-    float scale;
-    int l2norm;
-    PrepOut out;
-    const float* h0;
-    float* hT;
-    bf16* o;
-    int32_t* status;
-    int n_carry;
-    int stall;
-};
-
-// Bounded wait on a barrier of the carry CTA that also gives up at once when another role
-// has aborted.  Polls without suspending first (hand-offs on the serial chain are short).
-__device__ __forceinline__ bool fc_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
-                                        uint64_t timeout_ns = 2000000000ull) {
-    const uint32_t addr = tc::smem_u32(bar);
-    for (int i = 0; i < 2048; ++i)
-        if (tc::mbar_test_wait(addr, parity)) return true;
-    const uint64_t t0 = tc::globaltimer_ns();
-    while (true) {
-        for (int i = 0; i < 32; ++i)
-            if (tc::mbar_try_wait(addr, parity)) return true;
-        if (*abort) return false;
-        const uint64_t dt = tc::globaltimer_ns() - t0;
-        if (dt > timeout_ns) return false;
-        if (dt > 20000) __nanosleep(128);
-    }
-}
-
-// Wait (bounded) until a worker has published chunk-local item `flag`; gives up early if the
-// device status word reports a failure or the CTA aborted.
-__device__ __forceinline__ bool wait_flag(const int32_t* flag, const int32_t* status, const volatile int* abort) {
-    if (tc::ld_acquire_gpu(flag)) return true;
-    const uint64_t t0 = tc::globaltimer_ns();
-    while (true) {
-        for (int i = 0; i < 16; ++i)
-            if (tc::ld_acquire_gpu(flag)) return true;
-        if (*reinterpret_cast<const volatile int32_t*>(status) != 0 || *abort) return false;
-        const uint64_t dt = tc::globaltimer_ns() - t0;
-        if (dt > 2000000000ull) return false;
-        if (dt > 20000) __nanosleep(256);
-    }
-}
-
-__device__ __forceinline__ uint32_t pack_h2u(float lo, float hi) { return pack_h2(lo, hi); }
-
-// Walk the chains of carry CTA `cta` in order; f(n, h, bos, len, c0, nch) per chain.
-template <typename F>
-__device__ __forceinline__ void for_each_chain(const FusedArgs& fa, F&& f) {
-    const int n_chains = fa.n_seqs * fa.HV;
-    for (int j = blockIdx.x; j < n_chains; j += fa.n_carry) {
-        const int n = j / fa.HV, h = j - n * fa.HV;
-        const int64_t bos = fa.cu ? (int64_t)fa.cu[n] : (int64_t)n * fa.T;
-        const int64_t len = fa.cu ? (int64_t)fa.cu[n + 1] - fa.cu[n] : fa.T;
-        const int c0 = fa.chunk_off[n];
-        const int nch = fa.chunk_off[n + 1] - c0;
-        if (!f(n, h, bos, len, c0, nch)) break;
-    }
-}
-
-template <int G>
-__device__ void fused_carry(FcSmem& S, const CUtensorMap* tm_w, const CUtensorMap* tm_qh, const CUtensorMap* tm_kt,
-                            const CUtensorMap* tm_pt, const CUtensorMap* tm_u, const FusedArgs& fa, uint32_t tmem,
-                            int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int HV = fa.HV, HK = fa.HK;
-    const uint32_t tD1 = tmem + kFcD1, tD2 = tmem + kFcD2, tA1 = tmem + kFcA1, tA2 = tmem + kFcA2;
-    const volatile int* abort = &S.abort;
-
-    if (warp == 0) {
-        // ---------------- producer: flags, then the chunk's operands by TMA ----------------
-        if (lane != 0) return;
-        int it = 0;
-        for_each_chain(fa, [&](int n, int h, int64_t, int64_t, int c0, int nch) -> bool {
-            const int hk = h / G;
-            for (int c = 0; c < nch; ++c, ++it) {
-                const int st = it & 1, r = it >> 1;
-                FcStage& B = S.st[st];
-                const int cid = c0 + c;
-                // the step's two scalars first: the state epilogue of the step before needs them
-                // (entry it % 4 is free again: its reader finished step it - 3 before the stage
-                // this producer filled last was released)
-                bool ok = wait_flag(fa.out.flags + (size_t)cid * HK + hk, fa.status, abort);
-                if (ok) {
-                    const float* scg = fa.out.SC + ((size_t)cid * HV + h) * SC_FLOATS;
-                    S.nxt[it & 3][0] = scg[SC_GC];
-                    S.nxt[it & 3][1] = scg[SC_VMAX];
-                    tc::mbar_arrive(&S.scal[it & 3]);
-                }
-                ok = ok && (r == 0 || fc_wait(&S.empty[st], (uint32_t)((r - 1) & 1), abort));
-                if (!ok) {
-                    record_timeout(fa.status);
-                    S.abort = 1;
-                    return false;
-                }
-                tc::fence_async_global();   // the worker's stores, acquired above, before the copies
-                const int row = (cid * HV + h) * 64, qrow = (cid * HK + hk) * 64;
-                tc::mbar_expect_tx(&S.full[st], kFcTx);
-                tc::tma_load_2d(B.B1[0], tm_w, &S.full[st], 0, row);
-                tc::tma_load_2d(B.B1[1], tm_w, &S.full[st], 64, row);
-                tc::tma_load_2d(B.B1[0] + 8192, tm_qh, &S.full[st], 0, qrow);
-                tc::tma_load_2d(B.B1[1] + 8192, tm_qh, &S.full[st], 64, qrow);
-                tc::tma_load_2d(B.B2[0], tm_kt, &S.full[st], 0, row);
-                tc::tma_load_2d(B.B2[1], tm_kt, &S.full[st], 64, row);
-                tc::tma_load_2d(B.B2[2], tm_pt, &S.full[st], 0, row);
-                tc::tma_load_2d(B.U, tm_u, &S.full[st], 0, row * 2);   // U^T rows (chunk, head) * 128
-                tc::bulk_load(B.SC, fa.out.SC + ((size_t)cid * HV + h) * SC_FLOATS, SC_FLOATS * 4, &S.full[st]);
-                S.issued = it + 1;
-            }
-            return true;
-        });
-        return;
-    }
-    if (warp == 1) {
-        // ---------------- MMA issue ------------------------------------------------------------
-        if (lane != 0) return;
-        constexpr uint32_t idD1 = tc::idesc_f16(128, 128, 0, 0);   // B K-major
-        constexpr uint32_t idD2 = tc::idesc_f16(128, 192, 0, 1);   // B MN-major
-        int it = 0, d1_issued = 0, d2_issued = 0;
-        for_each_chain(fa, [&](int, int, int64_t, int64_t, int, int nch) -> bool {
-            for (int c = 0; c < nch; ++c, ++it) {
-                const int st = it & 1, r = it >> 1;
-                const FcStage& B = S.st[st];
-                bool ok = fc_wait(&S.full[st], (uint32_t)(r & 1), abort) &&
-                          fc_wait(&S.h_ready, (uint32_t)(it & 1), abort) &&
-                          fc_wait(&S.ofree1, (uint32_t)(it & 1), abort);
-                if (!ok) {
-                    record_timeout(fa.status);
-                    S.abort = 1;
-                    return false;
-                }
-                tc::tc_fence_after();
-                const uint32_t b1 = tc::smem_u32(B.B1[0]);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16_ts(tD1, tA1 + kk * 8, tc::desc_sw128(b1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                   idD1, kk > 0);
-                tc::mma_commit(&S.d1);
-                ++d1_issued;
-                ok = fc_wait(&S.d_ready, (uint32_t)(it & 1), abort) && fc_wait(&S.ofree2, (uint32_t)(it & 1), abort);
-                if (!ok) {
-                    record_timeout(fa.status);
-                    S.abort = 1;
-                    return false;
-                }
-                tc::tc_fence_after();
-                const uint64_t b2 = tc::desc_sw128(tc::smem_u32(B.B2[0]), 8192, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_f16_ts(tD2, tA2 + kk * 8, b2 + (uint64_t)((kk * 2048) >> 4), idD2, kk > 0);
-                tc::mma_commit(&S.d2);
-                tc::mma_commit(&S.empty[st]);
-                ++d2_issued;
-            }
-            return true;
-        });
-        if (S.abort) {   // products still running land before TMEM is released (at once if done)
-            if (d1_issued > 0) (void)tc::mbar_wait(&S.d1, (uint32_t)((d1_issued - 1) & 1), 50000000ull);
-            if (d2_issued > 0) (void)tc::mbar_wait(&S.d2, (uint32_t)((d2_issued - 1) & 1), 50000000ull);
-        }
-        return;
-    }
-    if (warp >= 4 && warp < 12) {
-        // ---------------- state epilogues: thread <-> (value column v, half hf) ------------------
-        // The fp32 state stays in registers: this thread holds H[k][v] for k in [64 hf, 64 hf + 64).
-        const int grp = warp & 3, v = grp * 32 + lane, hf = (warp - 4) >> 2;
-        const uint32_t lb = (uint32_t)(grp * 32) << 16;
-        const int wi = warp - 4;   // 0..7
-        int it = 0, ruse = 0;
-        bool ok = true;
-        float sc = 1.f, inv_sc = 1.f;
-        float H[64];
-        // max |H| over the 8 epilogue warps (one bar.red per call keeps the warps' decisions
-        // uniform: every warp learns whether any of them saw a failed wait)
-        auto block_max = [&](float m, bool& good) -> float {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            float* red = S.red[ruse & 1];
-            ++ruse;
-            if (lane == 0) red[wi] = m;
-            good = !tc::named_bar_any(2, 256, !good || S.abort);
-            float r = red[0];
-#pragma unroll
-            for (int i = 1; i < 8; ++i) r = fmaxf(r, red[i]);
-            return r;
-        };
-        // the data scale of step `in` from max |H| and that step's max |v|, then the fp16 operand
-        // H^T * sc into A1; returns with the operand complete in TMEM
-        auto publish_state = [&](int in, bool& good) {
-            float m = 0.f;
-#pragma unroll
-            for (int k = 0; k < 64; ++k) m = fmaxf(m, fabsf(H[k]));
-            good = fc_wait(&S.scal[in & 3], (uint32_t)((in >> 2) & 1), abort) && good;
-            m = block_max(m, good);
-            if (!good) return;
-            inv_sc = pow2_above(fmaxf(m, S.nxt[in & 3][1]));
-            sc = 1.f / inv_sc;
-            if (wi == 0 && lane == 0) S.scale[in & 3] = sc;
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) pk[j] = pack_h2u(H[32 * part + 2 * j] * sc, H[32 * part + 2 * j + 1] * sc);
-                tc::tmem_st16(tA1 + lb + 32 * hf + 16 * part, pk);
-            }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&S.h_ready);
-        };
-        for_each_chain(fa, [&](int n, int h, int64_t, int64_t, int, int nch) -> bool {
-            const size_t hrow = ((size_t)n * HV + h) * D * D;
-#pragma unroll
-            for (int k = 0; k < 64; ++k) H[k] = fa.h0 ? fa.h0[hrow + (size_t)(64 * hf + k) * D + v] : 0.f;
-            if (nch == 0) {   // nothing to carry: the final state is the initial one
-                if (fa.hT)
-#pragma unroll
-                    for (int k = 0; k < 64; ++k) fa.hT[hrow + (size_t)(64 * hf + k) * D + v] = H[k];
-                return true;
-            }
-            publish_state(it, ok);   // the chain's first operand, with the scale of its first chunk
-            if (!ok) return false;
-            for (int c = 0; c < nch; ++c, ++it) {
-                const int st = it & 1;
-                const FcStage& B = S.st[st];
-                // ---- Delta^T = U^T uinv - (W H)^T / sc, 32 tokens of this half -> A2 ----
-                ok = fc_wait(&S.full[st], (uint32_t)((it >> 1) & 1), abort) && ok;
-                ok = fc_wait(&S.d1, (uint32_t)(it & 1), abort) && ok;
-                tc::tc_fence_after();
-                const float gC = B.SC[SC_GC];
-                {
-                    float x[32];
-                    tc::tmem_ld32(tD1 + lb + 32 * hf, x);
-                    const float uinv = B.SC[SC_UINV];
-                    // row v of U^T, tokens 32 hf .. 32 hf + 31: 16-byte chunks 4 hf .. 4 hf + 3 of
-                    // the 128-byte row, at chunk ^ (v % 8) in the swizzled tile
-                    const uint4* urow = reinterpret_cast<const uint4*>(B.U + v * 128);
-                    uint4 u4[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) u4[q] = urow[(4 * hf + q) ^ (v & 7)];
-                    tc::tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const __half2* e = reinterpret_cast<const __half2*>(&u4[q]);
-#pragma unroll
-                        for (int p2 = 0; p2 < 4; ++p2) {
-                            const float2 uf = __half22float2(e[p2]);
-                            const int j = q * 4 + p2;
-                            const float d0 = uf.x * uinv - x[2 * j] * inv_sc;
-                            const float d1 = uf.y * uinv - x[2 * j + 1] * inv_sc;
-                            pk[j] = pack_h2u(d0 * sc, d1 * sc);
-                        }
-                    }
-                    tc::tmem_st16(tA2 + lb + 16 * hf, pk);
-                    tc::tmem_wait_st();
-                    tc::tc_fence_before();
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(&S.d_ready);
-                    tc::mbar_arrive(&S.empty[st]);   // this warp has read the stage's U and scalars
-                }
-                // ---- the new state H = gamma_C H + (K_tilde^T Delta) from D2 columns 0-127 ----
-                ok = fc_wait(&S.d2, (uint32_t)(it & 1), abort) && ok;
-                tc::tc_fence_after();
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    float y[32];
-                    tc::tmem_ld32(tD2 + lb + 64 * hf + 32 * part, y);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) H[32 * part + j] = fmaf(gC, H[32 * part + j], y[j] * inv_sc);
-                }
-                if (c == nch - 1) {   // chain done: the final state (no further step of this chain)
-                    // the step's one barrier, as in the other steps: every warp takes the same decision
-                    if (tc::named_bar_any(2, 256, !ok || S.abort)) {
-                        ok = false;
-                        return false;
-                    }
-                    if (fa.hT)
-#pragma unroll
-                        for (int k = 0; k < 64; ++k) fa.hT[hrow + (size_t)(64 * hf + k) * D + v] = H[k];
-                    continue;
-                }
-                publish_state(it + 1, ok);
-                if (!ok) return false;
-            }
-            return true;
-        });
-        if (!ok) {
-            record_timeout(fa.status);
-            S.abort = 1;
-        }
-        return;
-    }
-    if (warp >= 12) {
-        // ---------------- outputs: thread <-> value column v, all 64 tokens ------------------
-        const int grp = warp & 3, v = grp * 32 + lane;
-        const uint32_t lb = (uint32_t)(grp * 32) << 16;
-        if (lane == 0) {   // the output columns of D1 and D2 are free before the first step
-            tc::mbar_arrive(&S.ofree1);
-            tc::mbar_arrive(&S.ofree2);
-        }
-        int it = 0;
-        bool ok = true;
-        for_each_chain(fa, [&](int, int h, int64_t bos, int64_t len, int, int nch) -> bool {
-            for (int c = 0; c < nch; ++c, ++it) {
-                const int st = it & 1;
-                const FcStage& B = S.st[st];
-                const int64_t tok0 = bos + (int64_t)C * c;
-                const int64_t rem = len - (int64_t)C * c;
-                const int cn = (int)(rem < C ? rem : C);
-                ok = fc_wait(&S.full[st], (uint32_t)((it >> 1) & 1), abort) && ok;
-                ok = fc_wait(&S.d1, (uint32_t)(it & 1), abort) && ok;
-                tc::tc_fence_after();
-                float q[64];
-                tc::tmem_ld32(tD1 + lb + 64, q);
-                tc::tmem_ld32(tD1 + lb + 96, q + 32);
-                tc::tmem_wait_ld();
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&S.ofree1);
-                // (Q_hat H)^T * a: the row scalar a_t of each token, read now (the stage may go)
-#pragma unroll
-                for (int t = 0; t < 64; ++t) q[t] *= B.SC[t];
-                const float inv = 1.f / S.scale[it & 3];
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&S.empty[st]);   // this warp has read the stage's scalars
-                ok = fc_wait(&S.d2, (uint32_t)(it & 1), abort) && ok;
-                tc::tc_fence_after();
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float pd[32];
-                    tc::tmem_ld32(tD2 + lb + 128 + 32 * half, pd);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) q[32 * half + i] += pd[i];
-                }
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&S.ofree2);   // D2's output columns are read
-                bf16* ocol = fa.o + (size_t)(tok0 * HV + h) * D + v;
-#pragma unroll
-                for (int t = 0; t < 64; ++t)
-                    if (t < cn) ocol[(size_t)t * HV * D] = __float2bfloat16_rn(q[t] * inv);
-                if (!ok || S.abort) return false;
-            }
-            return true;
-        });
-        if (!ok) {
-            record_timeout(fa.status);
-            S.abort = 1;
-        }
-    }
-}
-
-template <int G>
-__global__ void __launch_bounds__(kFcThreads, 1)
-prefill_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
-                     const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_kt,
-                     const __grid_constant__ CUtensorMap tm_pt, const __grid_constant__ CUtensorMap tm_u,
-                     const FusedArgs fa) {
-    extern __shared__ uint8_t smem_raw[];
-    __shared__ uint32_t s_tmem;
-    __shared__ int s_failed;
-    uint8_t* base = align1024(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const bool carry = (int)blockIdx.x < fa.n_carry;
-    // an earlier stage of the call (the cu_seqlens check) failed: write nothing (read once, so
-    // that every thread of the CTA takes the same branch)
-    if (tid == 0) s_failed = *reinterpret_cast<volatile int32_t*>(fa.status) != 0;
-    if (warp == 0) {
-        tc::tmem_alloc(&s_tmem, 512);
-        tc::tmem_relinquish();
-    }
-    if (carry) {
-        FcSmem& S = *reinterpret_cast<FcSmem*>(base);
-        if (tid == 32) {
-            for (int i = 0; i < 2; ++i) {
-                tc::mbar_init(&S.full[i], 1);
-                tc::mbar_init(&S.empty[i], 1 + 8 + 4);   // MMA commit, 8 state warps (U), 4 output warps (scalars)
-            }
-            tc::mbar_init(&S.d1, 1);
-            tc::mbar_init(&S.d2, 1);
-            tc::mbar_init(&S.h_ready, 8);
-            tc::mbar_init(&S.d_ready, 8);
-            tc::mbar_init(&S.ofree1, 4);
-            tc::mbar_init(&S.ofree2, 4);
-            for (int i = 0; i < 4; ++i) tc::mbar_init(&S.scal[i], 1);
-            tc::fence_mbar_init();
-            S.abort = 0;
-            S.issued = 0;
-        }
-    } else if ((tid & 127) == 32) {
-        PrepSmem& S = *reinterpret_cast<PrepSmem*>(base + (tid >> 7) * kPrepSlot);
-        tc::mbar_init(&S.bar_load, 1);
-        tc::mbar_init(&S.bar_v, 1);
-        tc::mbar_init(&S.bar_mma, 1);
-        tc::fence_mbar_init();
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    if (s_failed) {
-    } else if (carry) {
-        fused_carry<G>(*reinterpret_cast<FcSmem*>(base), &tm_w, &tm_qh, &tm_kt, &tm_pt, &tm_u, fa, tmem, tid);
-    } else {
-        // ---------------- chunk-local workers: four per CTA, items in chunk order ----------------
-        const int wg = tid >> 7, wt = tid & 127;
-        PrepSmem& S = *reinterpret_cast<PrepSmem*>(base + wg * kPrepSlot);
-        const int worker = ((int)blockIdx.x - fa.n_carry) * 4 + wg;
-        const int n_workers = ((int)gridDim.x - fa.n_carry) * 4;
-        const int total = fa.chunk_off[fa.n_seqs] * fa.HK;
-        PrepPhases ph;
-        bool loaded = false;   // this item's K, Q copies were issued by the item before
-        for (int item = worker; item < total; item += n_workers) {
-            const bool failed = *reinterpret_cast<volatile int32_t*>(fa.status) != 0;
-            if (tc::named_bar_any(1 + wg, 128, failed)) break;   // every thread of the worker agrees
-            const int chunk = item / fa.HK, hk = item - chunk * fa.HK;
-            int n, cn, nn, ncn, nhk = -1;
-            int64_t s, ns = 0;
-            if (!locate_chunk(chunk, fa.chunk_off, fa.cu, fa.T, fa.n_seqs, n, s, cn)) break;
-            const int nitem = item + n_workers;
-            if (nitem < total) {
-                const int nchunk = nitem / fa.HK;
-                if (locate_chunk(nchunk, fa.chunk_off, fa.cu, fa.T, fa.n_seqs, nn, ns, ncn)) nhk = nitem - nchunk * fa.HK;
-            }
-            const bool ok = prep_item<G, true>(S, &tm_q, &tm_k, &tm_v, fa.g, fa.beta, chunk, hk, s, cn, fa.HV, fa.HK,
-                                               fa.scale, fa.l2norm, fa.out, fa.status,
-                                               fa.stall && chunk == 0 && hk == 0, tmem + 128 * wg, wt, 1 + wg, ph,
-                                               loaded, nhk, ns);
-            loaded = nhk >= 0;
-            if (!ok) {
-                loaded = false;
-                break;
-            }
-        }
-        // copies issued for an item that will not run land before the CTA leaves
-        if (loaded && wt == 0) (void)tc::mbar_wait(&S.bar_load, ph.load, 50000000ull);
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-    if (carry && tid == 0) {   // copies still in flight after an abort land before the CTA leaves:
-        FcSmem& S = *reinterpret_cast<FcSmem*>(base);   // the latest step issued on each stage
-        if (S.abort)
-            for (int k = S.issued - 2; k < S.issued; ++k)
-                if (k >= 0) (void)tc::mbar_wait(&S.full[k & 1], (uint32_t)((k >> 1) & 1), 50000000ull);
-    }
-    __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 512);
-}
-
-// ======================================================================================
 // host side
 // ======================================================================================
 struct TcLayout {
@@ -1818,29 +1165,6 @@ TcLayout tc_layout(int64_t n_tokens, int n_seqs, int HK, int HV) {
     L.off_p = round_up(L.off_u + rows * D * 2, 1024);
     L.off_qk = round_up(L.off_p + rows * 64 * 2, 1024);
     L.off_sc = round_up(L.off_qk + (size_t)L.max_chunks * HK * 128 * D * 2, 1024);
-    L.total = round_up(L.off_sc + (size_t)L.max_chunks * HV * SC_FLOATS * 4, 1024);
-    return L;
-}
-
-// Workspace of the fused launch: per (chunk, value head) W, U, P^T, K_tilde and scalars, per
-// (chunk, q/k head) Q_hat and a ready flag.
-struct FusedLayout {
-    int64_t max_chunks;
-    size_t off_chunk, off_flags, off_w, off_u, off_p, off_kt, off_q, off_sc, total;
-};
-
-FusedLayout fused_layout(int64_t n_tokens, int n_seqs, int HK, int HV) {
-    FusedLayout L;
-    L.max_chunks = (n_tokens + C - 1) / C + n_seqs;
-    const size_t rows = (size_t)L.max_chunks * HV * 64;
-    L.off_chunk = kStatusBytes;
-    L.off_flags = round_up(L.off_chunk + (size_t)(n_seqs + 1) * 4, 256);
-    L.off_w = round_up(L.off_flags + (size_t)L.max_chunks * HK * 4, 1024);
-    L.off_u = round_up(L.off_w + rows * D * 2, 1024);
-    L.off_p = round_up(L.off_u + rows * D * 2, 1024);
-    L.off_kt = round_up(L.off_p + rows * 64 * 2, 1024);
-    L.off_q = round_up(L.off_kt + rows * D * 2, 1024);
-    L.off_sc = round_up(L.off_q + (size_t)L.max_chunks * HK * 64 * D * 2, 1024);
     L.total = round_up(L.off_sc + (size_t)L.max_chunks * HV * SC_FLOATS * 4, 1024);
     return L;
 }
@@ -1880,131 +1204,10 @@ size_t prefill_tc_workspace_bytes(int64_t n_tokens, int n_seqs, int HK, int HV) 
     // TMA coordinates are 32-bit: token index, tile rows (chunk, head) * 64 and * 128
     const int64_t max_chunks = (n_tokens + C - 1) / C + n_seqs;
     if (n_tokens > INT32_MAX || max_chunks * HV * 64 > INT32_MAX || max_chunks * HK * 128 > INT32_MAX) return 0;
-    // one size for both launch forms (the fused one for the plain prefill, the two-kernel one
-    // for the output epilogue and the context-parallel segment)
-    const size_t a = tc_layout(n_tokens, n_seqs, HK, HV).total, b = fused_layout(n_tokens, n_seqs, HK, HV).total;
-    return a > b ? a : b;
+    return tc_layout(n_tokens, n_seqs, HK, HV).total;
 }
-
-namespace {
-int sm_count() {
-    static int cache[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (!cache[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        cache[dev] = n;
-    }
-    return cache[dev];
-}
-
-// The plain prefill (no output epilogue, no transition run) as one cooperative launch.
-cudaError_t launch_prefill_fused(const PrefillArgs& a, void* workspace, cudaStream_t s) {
-    const bool packed = a.cu != nullptr;
-    const int64_t n_tokens = packed ? a.T : (int64_t)a.n_seqs * a.T;
-    const FusedLayout L = fused_layout(n_tokens, a.n_seqs, a.HK, a.HV);
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    int32_t* chunk_off = reinterpret_cast<int32_t*>(ws + L.off_chunk);
-    int32_t* flags = reinterpret_cast<int32_t*>(ws + L.off_flags);
-    f16* W = reinterpret_cast<f16*>(ws + L.off_w);
-    f16* U = reinterpret_cast<f16*>(ws + L.off_u);
-    f16* P = reinterpret_cast<f16*>(ws + L.off_p);
-    f16* Kt = reinterpret_cast<f16*>(ws + L.off_kt);
-    f16* Q = reinterpret_cast<f16*>(ws + L.off_q);
-    float* SC = reinterpret_cast<float*>(ws + L.off_sc);
-
-    chunk_table_kernel<<<1, 1024, 0, s>>>(a.cu, a.n_seqs, a.T, chunk_off, a.status, flags,
-                                          (int64_t)L.max_chunks * a.HK);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    count_launch();
-
-    CUtensorMap tq, tk, tv, tw, tqh, tkt, tpt, tu;
-    const cuuint64_t tok = (cuuint64_t)(n_tokens > 0 ? n_tokens : 1);
-    {
-        cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.HK, tok};
-        cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.HK * D * 2};
-        cuuint32_t box[3] = {64, 1, 64};
-        const void* qb = a.q ? a.q : workspace;
-        const void* kb = a.k ? a.k : workspace;
-        if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qb, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kb, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-    }
-    {
-        cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.HV, tok};
-        cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.HV * D * 2};
-        cuuint32_t box[3] = {64, 1, 64};
-        const void* vb = a.v ? a.v : workspace;
-        if (!make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, vb, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-    }
-    const cuuint64_t mc = (cuuint64_t)(L.max_chunks > 0 ? L.max_chunks : 1);
-    {
-        const cuuint64_t rows = mc * a.HV * 64;
-        cuuint64_t dims[2] = {(cuuint64_t)D, rows};
-        cuuint64_t str[1] = {(cuuint64_t)D * 2};
-        cuuint32_t box[2] = {64, 64};
-        if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, W, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&tkt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Kt, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-        // U^T: rows (chunk, value head) * 128 + value, 64 tokens each; one box is a whole tile
-        cuuint64_t udims[2] = {64, rows * 2};
-        cuuint64_t ustr[1] = {64 * 2};
-        cuuint32_t ubox[2] = {64, 128};
-        if (!make_map(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, U, 2, udims, ustr, ubox, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-        cuuint64_t pdims[2] = {64, rows};
-        cuuint64_t pstr[1] = {64 * 2};
-        if (!make_map(&tpt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, P, 2, pdims, pstr, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-        cuuint64_t qdims[2] = {(cuuint64_t)D, mc * a.HK * 64};
-        if (!make_map(&tqh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Q, 2, qdims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-    }
-
-    const int sms = sm_count();
-    if (sms < 2) return cudaErrorInvalidDevice;
-    const int n_chains = a.n_seqs * a.HV;
-    // carry CTAs: one per chain up to a quarter of the SMs (the chunk-local workers take the rest)
-    int n_carry = n_chains < sms / 4 ? n_chains : sms / 4;
-    if (n_carry < 1) n_carry = 1;
-    FusedArgs fa;
-    fa.g = a.g; fa.beta = a.beta; fa.cu = a.cu; fa.chunk_off = chunk_off; fa.T = a.T;
-    fa.n_seqs = a.n_seqs; fa.HK = a.HK; fa.HV = a.HV; fa.scale = a.scale; fa.l2norm = a.l2norm;
-    fa.out = PrepOut{W, U, P, Q, SC, Kt, flags};
-    fa.h0 = a.h0; fa.hT = a.hT; fa.o = (bf16*)a.o; fa.status = a.status; fa.n_carry = n_carry;
-    fa.stall = testing_stall_site() == GDN_STALL_PREFILL_PREP ? 1 : 0;
-
-    auto launch = [&](auto kern) -> cudaError_t {
-        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedSmemBytes);
-        if (err != cudaSuccess) return err;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)sms);
-        cfg.blockDim = dim3(kFcThreads);
-        cfg.dynamicSmemBytes = kFusedSmemBytes;
-        cfg.stream = s;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident at once: carry and workers meet
-        attr[0].val.cooperative = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tw, tqh, tkt, tpt, tu, fa);
-    };
-    const int G = a.HV / a.HK;
-    e = G == 1 ? launch(prefill_fused_kernel<1>) : G == 2 ? launch(prefill_fused_kernel<2>)
-                                                          : launch(prefill_fused_kernel<4>);
-    if (e != cudaSuccess) return e;
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    count_launch();
-    return cudaSuccess;
-}
-}  // namespace
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_t s) {
-    if (!a.z && !a.o_tr) return launch_prefill_fused(a, workspace, s);
     const bool packed = a.cu != nullptr;
     const int64_t n_tokens = packed ? a.T : (int64_t)a.n_seqs * a.T;
     const TcLayout L = tc_layout(n_tokens, a.n_seqs, a.HK, a.HV);
@@ -2016,7 +1219,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
     f16* QK = reinterpret_cast<f16*>(ws + L.off_qk);
     float* SC = reinterpret_cast<float*>(ws + L.off_sc);
 
-    chunk_table_kernel<<<1, 1024, 0, s>>>(a.cu, a.n_seqs, a.T, chunk_off, a.status, nullptr, 0);
+    chunk_table_kernel<<<1, 1024, 0, s>>>(a.cu, a.n_seqs, a.T, chunk_off, a.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();
@@ -2081,9 +1284,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
                 err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                            (int)cudaSharedmemCarveoutMaxShared);
             if (err != cudaSuccess) return err;
-            const PrepOut po{W, U, P, QK, SC, nullptr, nullptr};
             kern<<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T, a.n_seqs, a.HV,
-                                                   a.scale, a.l2norm, a.HK, po, a.status,
+                                                   a.scale, a.l2norm, a.HK, W, U, P, QK, SC, a.status,
                                                    testing_stall_site() == GDN_STALL_PREFILL_PREP ? 1 : 0);
             return cudaSuccess;
         };

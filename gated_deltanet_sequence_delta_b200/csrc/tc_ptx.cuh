@@ -135,18 +135,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     }
 }
 
-// ---- flags in global memory ----------------------------------------------------------
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-// Orders this thread's earlier (generic proxy) accesses of global memory, such as the load
-// that acquired a flag, before its later async-proxy accesses (tensor-map copies).
-__device__ __forceinline__ void fence_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // ---- proxies and TMEM ordering fences ------------------------------------------------
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -251,22 +239,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     tmem_ld16(taddr, v);
     tmem_ld16(taddr + 16, v + 16);
 }
-// 32 lanes x 16 / 32 consecutive 32-bit columns from registers: thread i of the warp writes
-// lane (base + i).  Complete (visible to later MMAs) after tmem_wait_st.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
-    tmem_st16(taddr, r);
-    tmem_st16(taddr + 16, r + 16);
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 // ---- MMA ------------------------------------------------------------------------------
 // D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 or fp16 inputs as the
 // instruction descriptor says, fp32 accumulate).
@@ -277,18 +249,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16: A is M = 128 lanes, K packed as pairs of
-// 16-bit values per 32-bit column (column j holds K elements 2j, 2j + 1), so a K step of 16
-// advances the A address by 8 columns.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 // Arrive once on `bar` when every MMA issued so far by this thread has completed.
