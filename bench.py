@@ -3,10 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdn|reference]
 
-One step = one pass of the whole prefill path over one batch: the gates
-(gdn_gates) and the chunked prefill (gdn_chunk_prefill) over the long-context
-workload B=1, T=32768, 16 q/k heads, 32 value heads, d=128, bf16, BT=64
-(synthetic, seeded).  The JSON line's ``value`` is prefill tokens/s over all
+One step = one pass of the whole prefill path over one batch: the chunked prefill
+with the gate prologue fused in (gdn_chunk_prefill_gated: raw a, b -> gates ->
+chunked gated delta rule) over the long-context workload B=1, T=32768, 16 q/k
+heads, 32 value heads, d=128, bf16, BT=64 (synthetic, seeded).  The JSON line's ``value`` is prefill tokens/s over all
 ranks.  The decode step (B=64, H=32, d=128, fp32 state, 1024 consecutive steps)
 is measured in the same run and reported under ``decode`` with its HBM roofline.
 
@@ -322,11 +322,12 @@ def bench_prefill(args, rank, world, dev, P, pk, dev_t, pinned, barrier, max_ove
     hT = torch.empty((1, HV, D, D), dtype=torch.float32, device=dev)
     ws = torch.empty(G.prefill_workspace_bytes(T, 1, HK, HV, D, D, BT, 1), dtype=torch.uint8, device=dev)
 
+    G.gdn_gates(a, b, A_log, dt_bias, g=g, beta=beta)   # for the output-epilogue leg below
+
     def prefill_step(evs=None):
-        G.gdn_gates(a, b, A_log, dt_bias, g=g, beta=beta)
         if evs is not None:
             evs[0].record()
-        G.gdn_chunk_prefill(q, k, v, g, beta, BT=BT, o=o, final_state=hT, workspace=ws)
+        G.gdn_chunk_prefill_gated(q, k, v, a, b, A_log, dt_bias, BT=BT, o=o, final_state=hT, workspace=ws)
         if evs is not None:
             evs[1].record()
 

@@ -5,7 +5,7 @@ is its thin binding.  Names are re-exported lazily so that ``inputs`` (the
 seeded workload generator) can be imported without loading torch or the
 library.
 """
-_BINDING = ("gdn_gates", "gdn_chunk_prefill", "gdn_chunk_prefill_outgate", "gdn_chunk_prefill_status",
+_BINDING = ("gdn_gates", "gdn_chunk_prefill", "gdn_chunk_prefill_gated", "gdn_chunk_prefill_outgate", "gdn_chunk_prefill_status",
             "gdn_conv_prefill", "gdn_conv_status", "gdn_cp_segment", "gdn_cp_combine", "gdn_cp_status", "gdn_decode_step", "gdn_decode_step_gated", "gdn_decode_step_fused",
             "gdn_decode_status", "gdn_chunk_prefill_host", "prefill_host_workspace_bytes",
             "GDNError", "GDNLibraryError", "prefill_workspace_bytes", "kernel_launches", "testing_stall",

@@ -46,6 +46,9 @@ _SIGS = {
     "gdn_chunk_prefill": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                            _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "gdn_chunk_prefill_status": ([_vp, _vp, ctypes.POINTER(_i32)], ctypes.c_int),
+    "gdn_chunk_prefill_gated": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64,
+                                 _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp],
+                                ctypes.c_int),
     "gdn_chunk_prefill_outgate": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                    _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp],
                                   ctypes.c_int),
@@ -217,6 +220,39 @@ def gdn_chunk_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, BT:
             _ptr(z), _ptr(norm_w), float(eps), _ptr(o), _ptr(final_state), _ptr(workspace), workspace.numel(),
             _stream())
         _check(st, "gdn_chunk_prefill_outgate")
+    return o, final_state
+
+
+def gdn_chunk_prefill_gated(q, k, v, a, b, A_log, dt_bias, initial_state=None, cu_seqlens=None, BT: int = 64,
+                            scale: float = 1.0, qk_l2norm: bool = True, output_final_state: bool = True,
+                            o=None, final_state=None, workspace=None):
+    """Chunked prefill with the gate prologue fused in: a, b [B, T, HV] (fp32 or bf16) and
+    A_log, dt_bias [HV] fp32 instead of g, beta (bit-identical to gdn_gates followed by
+    gdn_chunk_prefill).  Tensor-core shapes only.  Returns (o, final_state or None)."""
+    B, T, HK, Dk = q.shape
+    HV, Dv = v.shape[-2:]
+    if k.shape != q.shape or v.shape[:2] != (B, T) or a.shape != (B, T, HV) or b.shape != a.shape:
+        raise ValueError("inconsistent q/k/v/a/b shapes")
+    if k.dtype != q.dtype or v.dtype != q.dtype or b.dtype != a.dtype:
+        raise TypeError("q, k, v must share one dtype, and a, b another")
+    if A_log.dtype != torch.float32 or dt_bias.dtype != torch.float32:
+        raise TypeError("A_log, dt_bias must be fp32")
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    dcode = _dtype_code(q)
+    if o is None:
+        o = torch.empty((B, T, HV, Dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, HV, Dk, Dv), dtype=torch.float32, device=q.device)
+    need = prefill_workspace_bytes(B * T, N, HK, HV, Dk, Dv, BT, dcode)
+    if need == 0:
+        _check(4, "gdn_chunk_prefill_gated")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().gdn_chunk_prefill_gated(
+        _ptr(q), _ptr(k), _ptr(v), dcode, _ptr(a), _ptr(b), _dtype_code(a), _ptr(A_log), _ptr(dt_bias),
+        _ptr(initial_state), _ptr(cu_seqlens), B, T, N, HK, HV, Dk, Dv, BT, float(scale), int(bool(qk_l2norm)),
+        _ptr(o), _ptr(final_state), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, "gdn_chunk_prefill_gated")
     return o, final_state
 
 

@@ -131,9 +131,20 @@ gdn_status prefill_check_sizes(gdn_dtype io_dtype, bool packed, int32_t B, int64
 }  // namespace gdn
 
 namespace {
-// gdn_chunk_prefill, with the output epilogue when z is given (tensor-core path only)
+// Raw gate inputs of gdn_chunk_prefill_gated (all null for the entry points that take g, beta).
+struct RawGates {
+    const void* a;
+    const void* b;
+    gdn_dtype ab_dtype;
+    const float* A_log;
+    const float* dt_bias;
+};
+
+// gdn_chunk_prefill, with the output epilogue when z is given (tensor-core path only) and the
+// gates formed in the kernel when g is null and gin.a is given (tensor-core path only)
 gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype io_dtype, const float* g,
-                        const float* beta, const float* initial_state, const int32_t* cu_seqlens, int32_t B,
+                        const float* beta, const RawGates& gin, const float* initial_state,
+                        const int32_t* cu_seqlens, int32_t B,
                         int64_t T, int32_t n_seqs, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
                         float scale, int32_t qk_l2norm, const void* z, const float* norm_w, float eps, void* o,
                         float* final_state, void* o_tr, float* final_tr, void* workspace, size_t workspace_bytes,
@@ -149,14 +160,18 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype i
     // ---- pointers ----------------------------------------------------------------
     if (!workspace) return GDN_ERR_WORKSPACE;
     if (workspace_bytes < need) return GDN_ERR_WORKSPACE;
-    if (n_tok > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
+    const bool raw = gin.a != nullptr || gin.b != nullptr;
+    if (raw && !(io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT))) return GDN_ERR_UNSUPPORTED;
+    if (raw && !dtype_ok(gin.ab_dtype)) return GDN_ERR_UNSUPPORTED;
+    if (n_tok > 0 && (!q || !k || !v || !o)) return GDN_ERR_NULL;
+    if (n_tok > 0 && (raw ? (!gin.a || !gin.b || !gin.A_log || !gin.dt_bias) : (!g || !beta))) return GDN_ERR_NULL;
     if (z && (!norm_w || !(eps >= 0.f))) return norm_w ? GDN_ERR_SHAPE : GDN_ERR_NULL;
     if ((z || o_tr) && !(io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT)))
         return GDN_ERR_UNSUPPORTED;
     if (o_tr && n_tok > 0 && !final_tr) return GDN_ERR_NULL;
     if (cu_seqlens == nullptr && n_tok == 0 && final_state == nullptr) return GDN_OK;
     const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, workspace, z, norm_w,
-                          o_tr, final_tr};
+                          o_tr, final_tr, gin.a, gin.b, gin.A_log, gin.dt_bias};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     // ---- aliasing ----------------------------------------------------------------
@@ -170,8 +185,11 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype i
     const Range rws{workspace, workspace_bytes};
     const Range rz{z, z ? (size_t)n_tok * HV * Dv * es : 0}, rnw{norm_w, z ? (size_t)Dv * 4 : 0};
     const Range rotr{o_tr, o_tr ? (size_t)n_tok * HV * Dv * es : 0}, rhtr{final_tr, o_tr ? state_bytes : 0};
+    const size_t eab = raw ? esize(gin.ab_dtype) : 0;
+    const Range rra{gin.a, (size_t)n_tok * HV * eab}, rrb{gin.b, (size_t)n_tok * HV * eab};
+    const Range rAl{gin.A_log, raw ? (size_t)HV * 4 : 0}, rdb{gin.dt_bias, raw ? (size_t)HV * 4 : 0};
     for (Range out : {ro, rhT, rws, rotr, rhtr}) {
-        for (Range in : {rq, rk, rv, rg, rb, rcu, rz, rnw})
+        for (Range in : {rq, rk, rv, rg, rb, rcu, rz, rnw, rra, rrb, rAl, rdb})
             if (overlap(out, in)) return GDN_ERR_ALIAS;
     }
     for (Range tr : {rotr, rhtr})
@@ -194,7 +212,9 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, gdn_dtype i
 
     gdn::PrefillArgs a;
     a.q = q; a.k = k; a.v = v; a.bf16 = io_dtype == GDN_BF16;
-    a.g = g; a.beta = beta; a.h0 = initial_state; a.cu = cu_seqlens;
+    a.g = raw ? nullptr : g; a.beta = raw ? nullptr : beta; a.h0 = initial_state; a.cu = cu_seqlens;
+    a.gates = raw ? gdn::DecodeGates{nullptr, nullptr, gin.a, gin.b, gin.ab_dtype == GDN_BF16, gin.A_log, gin.dt_bias}
+                  : gdn::DecodeGates{g, beta, nullptr, nullptr, false, nullptr, nullptr};
     a.T = T; a.n_seqs = n_seqs; a.HK = HK; a.HV = HV; a.Dk = Dk; a.Dv = Dv; a.BT = BT;
     a.scale = scale; a.l2norm = qk_l2norm ? 1 : 0; a.o = o; a.hT = final_state;
     a.z = z; a.norm_w = norm_w; a.eps = eps;
@@ -215,9 +235,21 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, gdn_dt
                              int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
                              float scale, int32_t qk_l2norm, void* o, float* final_state,
                              void* workspace, size_t workspace_bytes, void* stream) {
-    return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT,
-                        scale, qk_l2norm, nullptr, nullptr, 0.f, o, final_state, nullptr, nullptr, workspace,
+    return prefill_impl(q, k, v, io_dtype, g, beta, RawGates{}, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk,
+                        Dv, BT, scale, qk_l2norm, nullptr, nullptr, 0.f, o, final_state, nullptr, nullptr, workspace,
                         workspace_bytes, stream);
+}
+
+gdn_status gdn_chunk_prefill_gated(const void* q, const void* k, const void* v, gdn_dtype io_dtype, const void* a,
+                                   const void* b, gdn_dtype ab_dtype, const float* A_log, const float* dt_bias,
+                                   const float* initial_state, const int32_t* cu_seqlens, int32_t B, int64_t T,
+                                   int32_t n_seqs, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, int32_t BT,
+                                   float scale, int32_t qk_l2norm, void* o, float* final_state, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    if (!a || !b) return GDN_ERR_NULL;
+    return prefill_impl(q, k, v, io_dtype, nullptr, nullptr, RawGates{a, b, ab_dtype, A_log, dt_bias}, initial_state,
+                        cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT, scale, qk_l2norm, nullptr, nullptr, 0.f, o,
+                        final_state, nullptr, nullptr, workspace, workspace_bytes, stream);
 }
 
 gdn_status gdn_chunk_prefill_outgate(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
@@ -227,8 +259,8 @@ gdn_status gdn_chunk_prefill_outgate(const void* q, const void* k, const void* v
                                      int32_t qk_l2norm, const void* z, const float* norm_w, float eps, void* o,
                                      float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
     if (!z) return GDN_ERR_NULL;
-    return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT,
-                        scale, qk_l2norm, z, norm_w, eps, o, final_state, nullptr, nullptr, workspace,
+    return prefill_impl(q, k, v, io_dtype, g, beta, RawGates{}, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk,
+                        Dv, BT, scale, qk_l2norm, z, norm_w, eps, o, final_state, nullptr, nullptr, workspace,
                         workspace_bytes, stream);
 }
 
@@ -239,8 +271,8 @@ gdn_status gdn_cp_segment(const void* q, const void* k, const void* v, gdn_dtype
                           void* workspace, size_t workspace_bytes, void* stream) {
     if (!c) return GDN_ERR_NULL;
     if (Dk != Dv) return GDN_ERR_UNSUPPORTED;
-    return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk, Dv, BT,
-                        scale, qk_l2norm, nullptr, nullptr, 0.f, o, final_state, c, transition, workspace,
+    return prefill_impl(q, k, v, io_dtype, g, beta, RawGates{}, initial_state, cu_seqlens, B, T, n_seqs, HK, HV, Dk,
+                        Dv, BT, scale, qk_l2norm, nullptr, nullptr, 0.f, o, final_state, c, transition, workspace,
                         workspace_bytes, stream);
 }
 

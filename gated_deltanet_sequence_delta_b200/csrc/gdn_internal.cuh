@@ -59,8 +59,9 @@ cudaError_t launch_gates(const void* a, const void* b, bool ab_bf16, const float
                          const float* dt_bias, int64_t n_tokens, int HV, float* g, float* beta,
                          cudaStream_t s);
 
-// Where a decode step takes its gates from: g, beta [B, HV] as given, or (g == nullptr)
-// formed in the kernel from a, b [B, HV] (bf16 or fp32) and A_log, dt_bias [HV].
+// Where a kernel takes its gates from: g, beta [rows, HV] as given, or (g == nullptr) formed
+// in the kernel from a, b [rows, HV] (bf16 or fp32) and A_log, dt_bias [HV] (rows are the
+// decode step's sequences or the prefill's tokens).
 struct DecodeGates {
     const float* g;
     const float* beta;
@@ -70,7 +71,7 @@ struct DecodeGates {
     const float* A_log;
     const float* dt_bias;
 };
-__device__ __forceinline__ void decode_gates(const DecodeGates& G, int bh, int h, float& g, float& beta) {
+__device__ __forceinline__ void decode_gates(const DecodeGates& G, int64_t bh, int h, float& g, float& beta) {
     if (G.g) {
         g = G.g[bh];
         beta = G.beta[bh];
@@ -137,8 +138,9 @@ struct PrefillArgs {
     const void* k;
     const void* v;
     bool bf16;
-    const float* g;
+    const float* g;           // [tokens, HV], or null: gates formed in the kernel from `gates`
     const float* beta;
+    DecodeGates gates;        // the gate source (g, beta as above, or raw a, b with A_log, dt_bias)
     const float* h0;          // may be null
     const int32_t* cu;        // may be null (dense)
     int64_t T;                // tokens per sequence (dense) or total (packed)

@@ -172,6 +172,7 @@ gdn_status gdn_chunk_prefill_host(const void* q, const void* k, const void* v, g
     GDN_TRY(cudaMemcpyAsync(d_dtb, dt_bias, (size_t)HV * 4, cudaMemcpyHostToDevice, p.run));
     if (initial_state) GDN_TRY(cudaMemcpyAsync(d_state, initial_state, state_bytes, cudaMemcpyHostToDevice, p.run));
 
+    const bool fused_gates = io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT);
     const int64_t n_pieces = T > 0 ? (T + L.P - 1) / L.P : 0;
     for (int64_t i = 0; i < n_pieces; ++i) {
         const int sl = (int)(i & 1);
@@ -187,13 +188,20 @@ gdn_status gdn_chunk_prefill_host(const void* q, const void* k, const void* v, g
         // gates + prefill of piece i, the state carried in place
         GDN_TRY(cudaStreamWaitEvent(p.run, p.in_ready[sl], 0));
         if (i >= 2) GDN_TRY(cudaStreamWaitEvent(p.run, p.out_free[sl], 0));
-        gdn_status st = gdn_gates(ws + L.a[sl], ws + L.b[sl], ab_dtype, d_Alog, d_dtb, (int64_t)B * n, HV, d_g,
-                                  d_beta, p.run);
-        if (st != GDN_OK) return st;
-        st = gdn_chunk_prefill(ws + L.q[sl], ws + L.k[sl], ws + L.v[sl], io_dtype, d_g, d_beta,
-                               (i > 0 || initial_state) ? d_state : nullptr, nullptr, B, n, B, HK, HV, Dk, Dv, BT,
-                               scale, qk_l2norm, ws + L.o[sl], d_state, ws + L.prefill_ws, L.prefill_ws_bytes,
-                               p.run);
+        const float* h_in = (i > 0 || initial_state) ? d_state : nullptr;
+        gdn_status st;
+        if (fused_gates) {   // the tensor-core shapes form the gates inside the prefill
+            st = gdn_chunk_prefill_gated(ws + L.q[sl], ws + L.k[sl], ws + L.v[sl], io_dtype, ws + L.a[sl],
+                                         ws + L.b[sl], ab_dtype, d_Alog, d_dtb, h_in, nullptr, B, n, B, HK, HV, Dk,
+                                         Dv, BT, scale, qk_l2norm, ws + L.o[sl], d_state, ws + L.prefill_ws,
+                                         L.prefill_ws_bytes, p.run);
+        } else {
+            st = gdn_gates(ws + L.a[sl], ws + L.b[sl], ab_dtype, d_Alog, d_dtb, (int64_t)B * n, HV, d_g, d_beta, p.run);
+            if (st != GDN_OK) return st;
+            st = gdn_chunk_prefill(ws + L.q[sl], ws + L.k[sl], ws + L.v[sl], io_dtype, d_g, d_beta, h_in, nullptr, B, n,
+                                   B, HK, HV, Dk, Dv, BT, scale, qk_l2norm, ws + L.o[sl], d_state, ws + L.prefill_ws,
+                                   L.prefill_ws_bytes, p.run);
+        }
         if (st != GDN_OK) return st;
         GDN_TRY(cudaEventRecord(p.in_free[sl], p.run));
         GDN_TRY(cudaEventRecord(p.out_ready[sl], p.run));

@@ -318,8 +318,7 @@ __device__ __forceinline__ void store_tile_from_tmem(f16* __restrict__ dst, uint
 template <int G>
 __global__ void __launch_bounds__(128, 4)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
-                  const float* __restrict__ beta, const int32_t* __restrict__ cu,
+                  const __grid_constant__ CUtensorMap tm_v, const DecodeGates gs, const int32_t* __restrict__ cu,
                   const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HV, float scale,
                   int l2norm, int HK, f16* __restrict__ Wg, f16* __restrict__ Ug, f16* __restrict__ Pg,
                   f16* __restrict__ QKg, float* __restrict__ SCg, int32_t* __restrict__ status, int stall) {
@@ -363,13 +362,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc::tma_load_3d(kq + 8192, &tm_q, &S.bar_load, 0, hk, si);
         tc::tma_load_3d(kq + 16384 + 8192, &tm_q, &S.bar_load, 64, hk, si);
     }
+    // gates of token s + tid, value head h: read, or formed from the raw inputs (the formula of
+    // gdn_gates, so the two are bit-identical)
+    auto gate_of = [&](int h, float& gv, float& bv) {
+        gv = 0.f;
+        bv = 0.f;
+        if (tid < cn) decode_gates(gs, (s + tid) * HV + h, h, gv, bv);
+    };
     if (tid < 64) {   // gates of the group's first two value heads, under the TMA latency
 #pragma unroll
-        for (int gi = 0; gi < (G < 2 ? G : 2); ++gi) {
-            const int h = hk * G + gi;
-            S.ga[gi][tid] = tid < cn ? g[(s + tid) * HV + h] : 0.f;
-            S.ba[gi][tid] = tid < cn ? beta[(s + tid) * HV + h] : 0.f;
-        }
+        for (int gi = 0; gi < (G < 2 ? G : 2); ++gi) gate_of(hk * G + gi, S.ga[gi][tid], S.ba[gi][tid]);
     }
     bool ok = tc::mbar_wait(&S.bar_load, 0);
     if (__syncthreads_or(!ok)) goto abort;
@@ -460,10 +462,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 S.bt[tid] = S.ba[gi & 1][tid];
             }
             __syncthreads();
-            if (G > 2 && gi + 2 < G && tid < 64) {   // slot gi % 2 is read: value head gi + 2's gates
-                S.ga[gi & 1][tid] = tid < cn ? g[(s + tid) * HV + h + 2] : 0.f;
-                S.ba[gi & 1][tid] = tid < cn ? beta[(s + tid) * HV + h + 2] : 0.f;
-            }
+            if (G > 2 && gi + 2 < G && tid < 64)   // slot gi % 2 is read: value head gi + 2's gates
+                gate_of(h + 2, S.ga[gi & 1][tid], S.ba[gi & 1][tid]);
             if (tid >= 32 && tid < 64) S.G[tid] += S.G[31];
             __syncthreads();
             if (tid < 64) S.bgr[tid] = S.bt[tid] * expf(S.G[tid]);
@@ -1284,7 +1284,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
                 err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                            (int)cudaSharedmemCarveoutMaxShared);
             if (err != cudaSuccess) return err;
-            kern<<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.g, a.beta, a.cu, chunk_off, a.T, a.n_seqs, a.HV,
+            kern<<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.gates, a.cu, chunk_off, a.T, a.n_seqs, a.HV,
                                                    a.scale, a.l2norm, a.HK, W, U, P, QK, SC, a.status,
                                                    testing_stall_site() == GDN_STALL_PREFILL_PREP ? 1 : 0);
             return cudaSuccess;

@@ -152,6 +152,31 @@ GDN_API gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * gdn_chunk_prefill_gated -- gdn_chunk_prefill with the gate prologue fused in: instead of
+ * g and beta it takes the gate inputs and forms
+ *     g = -exp(A_log[h]) * softplus(a + dt_bias[h]),   beta = sigmoid(b)
+ * (the gate code of the "Gated DeltaNet ... Qwen3-next" page, section 2.1) per (token,
+ * value head) inside the chunk-local kernel, with the same arithmetic as gdn_gates, so the
+ * results are bit-identical to gdn_gates followed by gdn_chunk_prefill; g and beta are never
+ * written to memory.
+ *   a, b          [B, T, HV] (packed: [T, HV]), ab_dtype fp32 or bf16     (read)
+ *   A_log, dt_bias [HV] fp32                                             (read)
+ *   everything else as gdn_chunk_prefill, same workspace size.
+ * The tensor-core shapes only (bf16, Dk = Dv = 128, BT = 64, HV / HK in {1, 2, 4});
+ * others return UNSUPPORTED (use gdn_gates and gdn_chunk_prefill).
+ * Errors: those of gdn_chunk_prefill; ALIAS also for outputs over a, b, A_log, dt_bias.
+ */
+GDN_API gdn_status gdn_chunk_prefill_gated(const void* q, const void* k, const void* v, gdn_dtype io_dtype,
+                             const void* a, const void* b, gdn_dtype ab_dtype,
+                             const float* A_log, const float* dt_bias,
+                             const float* initial_state, const int32_t* cu_seqlens,
+                             int32_t B, int64_t T, int32_t n_seqs,
+                             int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                             int32_t BT, float scale, int32_t qk_l2norm,
+                             void* o, float* final_state,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * gdn_chunk_prefill_outgate -- gdn_chunk_prefill with the output epilogue fused into the
  * output store: each output row of a value head (Dv values) becomes
  *     o * rsqrt(mean(o^2) + eps) * (1 + norm_w) * sigmoid(z)
@@ -321,7 +346,8 @@ GDN_API gdn_status gdn_chunk_prefill_static_ws(const void* q, const void* k, con
 
 /*
  * gdn_chunk_prefill_host -- gdn_gates followed by gdn_chunk_prefill for inputs and outputs
- * that live in HOST memory.  The sequences are streamed through the GPU in pieces of
+ * that live in HOST memory (on the tensor-core shapes, gdn_chunk_prefill_gated: the gates
+ * formed inside the prefill, bit for bit the same).  The sequences are streamed through the GPU in pieces of
  * `piece_tokens` tokens (a multiple of BT): the host -> device copies of one piece, the
  * kernels of the previous piece and the device -> host copies of the one before overlap
  * on three library-owned streams with two buffer slots each way, and the state is carried

@@ -307,3 +307,23 @@ def test_static_scratch_entry_point_reports_sizes_like_the_workspace_one(L):
         assert want != 0, kw
         assert static(**kw) == want, (kw, static(**kw), want)
     assert static(HK=2, HV=3) == 2   # GDN_ERR_SHAPE, as gdn_chunk_prefill
+
+
+def test_prefill_gated_validation(L):
+    def call(**kw):
+        a = dict(q=A, k=A + 64 * MB, v=A + 128 * MB, io=1, ga=A + 192 * MB, gb=A + 200 * MB, ab=0, Al=A + 208 * MB,
+                 dtb=A + 209 * MB, h0=None, cu=None, B=1, T=128, N=1, HK=2, HV=4, Dk=128, Dv=128, BT=64,
+                 o=A + 256 * MB, hT=A + 384 * MB, ws=A + 448 * MB, ws_bytes=1 << 30)
+        a.update(kw)
+        return L.gdn_chunk_prefill_gated(a["q"], a["k"], a["v"], a["io"], a["ga"], a["gb"], a["ab"], a["Al"], a["dtb"],
+                                         a["h0"], a["cu"], a["B"], a["T"], a["N"], a["HK"], a["HV"], a["Dk"], a["Dv"],
+                                         a["BT"], 1.0, 1, a["o"], a["hT"], a["ws"], a["ws_bytes"], None)
+    assert call(ga=None) == 1                  # NULL gate input
+    assert call(Al=None) == 1
+    assert call(HV=3) == 2                     # HV % HK
+    assert call(Dk=64, Dv=64) == 4             # not a tensor-core shape
+    assert call(io=0) == 4                     # fp32 io: the CUDA-core path has no fused gates
+    assert call(ab=7) == 4                     # unknown gate dtype
+    assert call(ga=A + 192 * MB + 4) == 3      # misaligned
+    assert call(o=A + 192 * MB) == 5           # output over a gate input
+    assert call(ws_bytes=16) == 6
