@@ -509,8 +509,10 @@ def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, 
     k1 = torch.cuda.Event(enable_timing=True)
     w0 = time.time()
     k0.record()
+    torch.cuda.nvtx.range_push("decode_b64")   # (lets a profiler pick a launch from the middle of this run)
     for i in range(n_dec):
         G.gdn_decode_step(dq, dk, dv, dg, dbeta, state, o=do)
+    torch.cuda.nvtx.range_pop()
     k1.record()
     barrier()
     clocks.window(w0, time.time())
@@ -556,6 +558,49 @@ def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, 
     clocks.window(w0, time.time())
     fused_launches = G.kernel_launches() - nc0
     fused_ms = max_over_ranks(c0.elapsed_time(c1) / n_dec)
+    # the same step with the output epilogue (zero-centred RMSNorm times 1 + w, sigmoid(z)) before
+    # the store: gdn_decode_step_fused_outgate
+    zring = [dev_t(fs.out_z(s_)).view(ds.B, ds.HV, ds.Dv) for s_ in range(8)]
+    nwd = dev_t(fs.out_w())
+
+    def fused_outgate_step(i):
+        x, a_, b_ = fring[i % len(fring)]
+        G.gdn_decode_step_fused(x, cw, cst[i % 2], a_, b_, dA, dbias, state, HK=ds.HK, conv_act=1, o=do,
+                                conv_state_out=cst[(i + 1) % 2], outgate=(zring[i % len(zring)], nwd, 1e-6))
+
+    for i in range(3):
+        fused_outgate_step(i)
+    barrier()
+    c0.record()
+    for i in range(n_dec):
+        fused_outgate_step(i)
+    c1.record()
+    barrier()
+    fused_og_ms = max_over_ranks(c0.elapsed_time(c1) / n_dec)
+    del zring
+    # a state twice the size of L2: B = 128 (256 MiB), the step alone (gates precomputed), so
+    # that the HBM figure cannot rest on a state that stays in the 126 MB L2
+    big = I.decode(B=2 * DECODE["B"], H=DECODE["H"], D=DECODE["D"], seed=replica_seed(5, rank))
+    bstate = dev_t(big.state0)
+    bq, bk, bv, ba_, bb_ = big.step(0)
+    bq, bk, bv = dev_t(bq), dev_t(bk), dev_t(bv)
+    bg, bbeta = G.gdn_gates(dev_t(ba_), dev_t(bb_), dev_t(big.A_log), dev_t(big.dt_bias))
+    bo = torch.empty((big.B, big.HV, big.Dv), dtype=torch.bfloat16, device=dev)
+    n_big = 256
+    for _ in range(3):
+        G.gdn_decode_step(bq, bk, bv, bg, bbeta, bstate, o=bo)
+    barrier()
+    c0.record()
+    torch.cuda.nvtx.range_push("decode_b128")
+    for _ in range(n_big):
+        G.gdn_decode_step(bq, bk, bv, bg, bbeta, bstate, o=bo)
+    torch.cuda.nvtx.range_pop()
+    c1.record()
+    barrier()
+    big_ms = max_over_ranks(c0.elapsed_time(c1) / n_big)
+    big_bytes = decode_bytes_per_step(big.B, big.HK, big.HV, big.Dk, big.Dv)
+    big_gbs = big_bytes / (big_ms * 1e-3) / 1e9
+    del bstate
     fbytes = (2 * ds.B * ds.HV * ds.Dk * ds.Dv * 4          # state in and out
               + ds.B * fs.C * 2 + 2 * ds.B * fs.C * 3 * 4   # x (bf16), convolution state in and out
               + fs.C * 16 + ds.B * ds.HV * (2 * 4 + ds.Dv * 2) + 2 * ds.HV * 4)   # weights, a, b, o, A_log, dt_bias
@@ -572,6 +617,14 @@ def bench_decode(args, rank, world, dev, P, pk, dev_t, barrier, max_over_ranks, 
                                    "gates and update in one launch per step",
                            "ms_per_step": fused_ms, "steps_per_s": world * 1e3 / fused_ms, "bytes_per_step": fbytes,
                            "achieved_gbs": fgbs, "frac": fgbs / P["hbm_gbs"], "gpu_launches": fused_launches},
+            "fused_outgate_step": {"what": "gdn_decode_step_fused_outgate: the step from raw projections with the "
+                                           "output epilogue (zero-centred RMSNorm x (1 + w), sigmoid(z), eps 1e-6) "
+                                           "before the store",
+                                   "ms_per_step": fused_og_ms, "steps_per_s": world * 1e3 / fused_og_ms,
+                                   "vs_fused_step_us": (fused_og_ms - fused_ms) * 1e3},
+            "state_2x_l2": {"what": "gdn_decode_step alone on B=128 (state 256 MiB, twice the L2), 256 steps",
+                            "ms_per_step": big_ms, "bytes_per_step": big_bytes, "achieved_gbs": big_gbs,
+                            "frac": big_gbs / P["hbm_gbs"]},
             "gated_step": {"what": "gdn_decode_step_gated: gates formed in the decode kernel, one launch per step",
                            "ms_per_step": gated_ms, "steps_per_s": world * 1e3 / gated_ms,
                            "achieved_gbs": ggbs, "frac": ggbs / P["hbm_gbs"], "gpu_launches": gated_launches},

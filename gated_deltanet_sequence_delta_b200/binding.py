@@ -64,6 +64,9 @@ _SIGS = {
                         _vp], ctypes.c_int),
     "gdn_decode_step_fused": ([_vp, ctypes.c_int, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_int, _vp, _vp, _vp,
                                _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp], ctypes.c_int),
+    "gdn_decode_step_fused_outgate": ([_vp, ctypes.c_int, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_int, _vp, _vp,
+                                       _vp, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _f32, _vp, _vp],
+                                      ctypes.c_int),
     "gdn_chunk_prefill_host_workspace_bytes": ([_i32, _i64, _i32, _i32, _i32, _i32, _i32, ctypes.c_int,
                                                 ctypes.c_int, _i64], _sz),
     "gdn_chunk_prefill_host": ([_vp, _vp, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _i32, _i64,
@@ -354,10 +357,12 @@ def gdn_chunk_prefill_host(q, k, v, a, b, A_log, dt_bias, initial_state=None, BT
 
 
 def gdn_decode_step_fused(x, conv_w, conv_state_in, a, b, A_log, dt_bias, state, HK: int, conv_act: int = 1,
-                          scale: float = 1.0, qk_l2norm: bool = True, conv_state_out=None, o=None):
+                          scale: float = 1.0, qk_l2norm: bool = True, conv_state_out=None, o=None, outgate=None):
     """The decode step from raw projections: x [B, C] (C = 2 HK Dk + HV Dv, q | k | v),
     conv_w [C, 4], conv_state_in [B, 3, C] (tap-major, oldest first); a, b [B, HV];
-    A_log, dt_bias [HV]; state [B, HV, Dk, Dv] updated in place.
+    A_log, dt_bias [HV]; state [B, HV, Dk, Dv] updated in place.  With outgate = (z, norm_w,
+    eps), z [B, HV, Dv] like o and norm_w [Dv] fp32, each output row becomes
+    o * rsqrt(mean(o^2) + eps) * (1 + norm_w) * sigmoid(z) (gdn_decode_step_fused_outgate).
     Returns (o [B, HV, Dv], conv_state_out [B, 3, C])."""
     B, HV, Dk, Dv = state.shape
     C = 2 * HK * Dk + HV * Dv
@@ -369,11 +374,22 @@ def gdn_decode_step_fused(x, conv_w, conv_state_in, a, b, A_log, dt_bias, state,
         conv_state_out = torch.empty_like(conv_state_in)
     if o is None:
         o = torch.empty((B, HV, Dv), dtype=x.dtype, device=x.device)
-    st = lib().gdn_decode_step_fused(_ptr(x), _dtype_code(x), _ptr(conv_w), _ptr(conv_state_in),
-                                     _ptr(conv_state_out), int(conv_act), _ptr(a), _ptr(b), _dtype_code(a),
-                                     _ptr(A_log), _ptr(dt_bias), _ptr(state), B, HK, HV, Dk, Dv, float(scale),
-                                     int(bool(qk_l2norm)), _ptr(o), _stream())
-    _check(st, "gdn_decode_step_fused")
+    if outgate is None:
+        st = lib().gdn_decode_step_fused(_ptr(x), _dtype_code(x), _ptr(conv_w), _ptr(conv_state_in),
+                                         _ptr(conv_state_out), int(conv_act), _ptr(a), _ptr(b), _dtype_code(a),
+                                         _ptr(A_log), _ptr(dt_bias), _ptr(state), B, HK, HV, Dk, Dv, float(scale),
+                                         int(bool(qk_l2norm)), _ptr(o), _stream())
+        _check(st, "gdn_decode_step_fused")
+    else:
+        z, norm_w, eps = outgate
+        if z.shape != o.shape or z.dtype != x.dtype or norm_w.shape != (Dv,) or norm_w.dtype != torch.float32:
+            raise ValueError("z must be shaped and typed like o; norm_w fp32 [Dv]")
+        st = lib().gdn_decode_step_fused_outgate(_ptr(x), _dtype_code(x), _ptr(conv_w), _ptr(conv_state_in),
+                                                 _ptr(conv_state_out), int(conv_act), _ptr(a), _ptr(b),
+                                                 _dtype_code(a), _ptr(A_log), _ptr(dt_bias), _ptr(state), B, HK, HV,
+                                                 Dk, Dv, float(scale), int(bool(qk_l2norm)), _ptr(z), _ptr(norm_w),
+                                                 float(eps), _ptr(o), _stream())
+        _check(st, "gdn_decode_step_fused_outgate")
     return o, conv_state_out
 
 

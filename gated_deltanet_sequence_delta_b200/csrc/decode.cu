@@ -177,6 +177,7 @@ struct StagedSmem {
     ConvSlot cv[CONV ? kSStages : 1];
     float delta[kSD];
     float dot[4];
+    float osq[4];   // output epilogue: per warp of the row, its part of sum(o^2)
     uint64_t full[kSStages], empty[kSStages];
 };
 template <bool CONV>
@@ -190,11 +191,23 @@ __device__ __forceinline__ float ld_raw(const uint8_t* p, int i) {
 // CONV: q, k, v are not read from memory but formed from the raw projections by the
 // convolution prologue (threads 0-383, one channel each: q, k, v rows of this item), kept
 // in the slot as fp32.
-template <typename IO, bool CONV>
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 from the hardware tanh (one special-function op, about
+// 2^-11 relative error): an absolute gate error below 2^-12
+__device__ __forceinline__ float sigmoid_tanh(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
+
+// OUTG (with CONV only): the output epilogue of the Qwen3-next page (section 3.2: a
+// zero-centred RMSNorm, weight stored as w with the scale 1 + w) and the sigmoid output gate of
+// the GDN resource-allocation page, on each output row before the store.
+template <typename IO, bool CONV, bool OUTG = false>
 __global__ void __launch_bounds__(kSThreads, 1)
 decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                      const DecodeConv conv, const DecodeGates gates, float* __restrict__ state, int n_items,
-                     int HK, int HV, float scale, int l2norm, IO* __restrict__ o, int stall) {
+                     int HK, int HV, float scale, int l2norm, IO* __restrict__ o, int stall,
+                     const DecodeOutGate og) {
     using QT = typename std::conditional<CONV, float, IO>::type;   // element type of the q, k, v rows
     constexpr int CPL = kSD / 32;   // 4 columns per lane
     constexpr uint32_t kRowBytes = kSD * sizeof(IO);
@@ -265,6 +278,7 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
         const int bh_ = item, b_ = bh_ / HV, h_ = bh_ - b_ * HV, hk_ = h_ / (HV / HK);
         return cseg < 2 ? (int64_t)cseg * HK * kSD + (int64_t)hk_ * kSD + cd : (int64_t)2 * HK * kSD + (int64_t)h_ * kSD + cd;
     };
+    const float wj = OUTG && tid < kSD ? 1.f + og.w[tid] : 1.f;   // (1 + w) of output column tid
     float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);   // this item's taps (weights), an item ahead
     if (CONV && tid < 3 * kSD && n_mine > 0) cw = *reinterpret_cast<const float4*>(conv.w + conv_channel(blockIdx.x) * 4);
     for (int i = 0; i < n_mine; ++i) {
@@ -273,6 +287,8 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
         StagedSlot& B = S.st[st];
         float gv, bt;
         decode_gates(gates, bh, bh % HV, gv, bt);   // issued before the wait
+        float zj = 0.f;   // the gate input of output column tid, also issued before the wait
+        if (OUTG && tid < kSD) zj = load_elem(reinterpret_cast<const IO*>(og.z), (int64_t)bh * kSD + tid);
         const float alpha = expf(gv);
         const bool ok = tc::mbar_wait(&S.full[st], r & 1);
         if (tc::named_bar_any(1, kSWarps * 32, !ok)) {   // uniform decision to stop
@@ -347,8 +363,17 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
                 sq += red_q[w * kSD + j];
             }
             const float delta = bt * (ld_raw<QT>(B.v, j) - alpha * su * rk);
-            store_elem(o, (int64_t)bh * kSD + j, scale * (alpha * (sq * rq) + delta * kq));
+            const float oj = scale * (alpha * (sq * rq) + delta * kq);
             S.delta[j] = delta;
+            if (!OUTG) {
+                store_elem(o, (int64_t)bh * kSD + j, oj);
+            } else {   // the row's mean square over its 128 values: these four warps, one barrier
+                const float ss = warp_sum(oj * oj);
+                if (lane == 0) S.osq[warp] = ss;
+                tc::named_bar(2, kSD);
+                const float ms = (S.osq[0] + S.osq[1] + S.osq[2] + S.osq[3]) * (1.f / kSD);
+                store_elem(o, (int64_t)bh * kSD + j, oj * rsqrtf(ms + og.eps) * wj * sigmoid_tanh(zj));
+            }
         }
         tc::named_bar(1, kSWarps * 32);
         // H' = alpha H + k_hat delta^T, written back in place
@@ -392,22 +417,22 @@ int staged_grid() {
     return sms[dev];
 }
 
-template <typename IO, bool CONV>
+template <typename IO, bool CONV, bool OUTG = false>
 cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, const DecodeConv& conv,
                                  const DecodeGates& gates, float* state, int B, int HK, int HV, float scale,
-                                 int l2norm, void* o, cudaStream_t s) {
+                                 int l2norm, void* o, cudaStream_t s, const DecodeOutGate& og = DecodeOutGate{}) {
     const int n_items = B * HV;
     const int sms = staged_grid();
     if (sms <= 0) return cudaErrorInvalidDevice;
     constexpr size_t smem = staged_smem_bytes<CONV>();
     static_assert(smem <= 227 * 1024, "staged decode: shared memory over the per-block limit");
-    cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<IO, CONV>,
+    cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<IO, CONV, OUTG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = n_items < sms ? n_items : sms;
-    decode_staged_kernel<IO, CONV><<<grid, kSThreads, smem, s>>>(
+    decode_staged_kernel<IO, CONV, OUTG><<<grid, kSThreads, smem, s>>>(
         (const IO*)q, (const IO*)k, (const IO*)v, conv, gates, state, n_items, HK, HV, scale, l2norm, (IO*)o,
-        testing_stall_site() == GDN_STALL_DECODE ? 1 : 0);
+        testing_stall_site() == GDN_STALL_DECODE ? 1 : 0, og);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
@@ -449,8 +474,14 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, bool bf16
 }
 
 cudaError_t launch_decode_conv(bool bf16, const DecodeConv& conv, const DecodeGates& gates, float* state, int B,
-                               int HK, int HV, float scale, int l2norm, void* o, cudaStream_t s) {
+                               int HK, int HV, float scale, int l2norm, void* o, const DecodeOutGate& og,
+                               cudaStream_t s) {
     if (B == 0) return cudaSuccess;
+    if (og.z)
+        return bf16 ? launch_decode_staged<__nv_bfloat16, true, true>(nullptr, nullptr, nullptr, conv, gates, state, B,
+                                                                      HK, HV, scale, l2norm, o, s, og)
+                    : launch_decode_staged<float, true, true>(nullptr, nullptr, nullptr, conv, gates, state, B, HK, HV,
+                                                              scale, l2norm, o, s, og);
     return bf16 ? launch_decode_staged<__nv_bfloat16, true>(nullptr, nullptr, nullptr, conv, gates, state, B, HK, HV,
                                                             scale, l2norm, o, s)
                 : launch_decode_staged<float, true>(nullptr, nullptr, nullptr, conv, gates, state, B, HK, HV, scale,

@@ -338,11 +338,15 @@ gdn_status gdn_decode_step_gated(const void* q, const void* k, const void* v, gd
                                           qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
 }
 
-gdn_status gdn_decode_step_fused(const void* x, gdn_dtype io_dtype, const float* conv_w, const float* conv_state_in,
-                                 float* conv_state_out, int32_t conv_act, const void* a, const void* b,
-                                 gdn_dtype ab_dtype, const float* A_log, const float* dt_bias, float* state,
-                                 int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, float scale,
-                                 int32_t qk_l2norm, void* o, void* stream) {
+}  // extern "C"
+
+namespace {
+// gdn_decode_step_fused, with the output epilogue when og.z is given
+gdn_status decode_fused_impl(const void* x, gdn_dtype io_dtype, const float* conv_w, const float* conv_state_in,
+                             float* conv_state_out, int32_t conv_act, const void* a, const void* b,
+                             gdn_dtype ab_dtype, const float* A_log, const float* dt_bias, float* state, int32_t B,
+                             int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm,
+                             const gdn::DecodeOutGate& og, void* o, void* stream) {
     if (B < 0 || HK <= 0 || HV <= 0 || Dk <= 0 || Dv <= 0 || HV % HK != 0) return GDN_ERR_SHAPE;
     if (!dtype_ok(io_dtype) || !dtype_ok(ab_dtype) || Dk != 128 || Dv != 128 || (conv_act != 0 && conv_act != 1))
         return GDN_ERR_UNSUPPORTED;
@@ -363,10 +367,43 @@ gdn_status gdn_decode_step_fused(const void* x, gdn_dtype io_dtype, const float*
         for (Range in : {rx, rw, rci, ra, rb, rA, rd})
             if (overlap(out, in)) return GDN_ERR_ALIAS;
     if (overlap(rs, ro) || overlap(rs, rco) || overlap(ro, rco)) return GDN_ERR_ALIAS;
+    if (og.z) {   // the output epilogue's inputs
+        if (!og.w) return GDN_ERR_NULL;
+        if (!(og.eps >= 0.f)) return GDN_ERR_SHAPE;
+        if (!aligned16(og.z) || !aligned16(og.w)) return GDN_ERR_ALIGN;
+        const Range rz{og.z, (size_t)B * HV * Dv * es}, rw2{og.w, (size_t)Dv * 4};
+        for (Range out : {rs, ro, rco})
+            for (Range in : {rz, rw2})
+                if (overlap(out, in)) return GDN_ERR_ALIAS;
+    }
     const gdn::DecodeGates gates{nullptr, nullptr, a, b, ab_dtype == GDN_BF16, A_log, dt_bias};
     const gdn::DecodeConv conv{x, conv_w, conv_state_in, conv_state_out, conv_act};
     return cuda_status(gdn::launch_decode_conv(io_dtype == GDN_BF16, conv, gates, state, B, HK, HV, scale,
-                                               qk_l2norm ? 1 : 0, o, (cudaStream_t)stream));
+                                               qk_l2norm ? 1 : 0, o, og, (cudaStream_t)stream));
+}
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_decode_step_fused(const void* x, gdn_dtype io_dtype, const float* conv_w, const float* conv_state_in,
+                                 float* conv_state_out, int32_t conv_act, const void* a, const void* b,
+                                 gdn_dtype ab_dtype, const float* A_log, const float* dt_bias, float* state,
+                                 int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv, float scale,
+                                 int32_t qk_l2norm, void* o, void* stream) {
+    return decode_fused_impl(x, io_dtype, conv_w, conv_state_in, conv_state_out, conv_act, a, b, ab_dtype, A_log,
+                             dt_bias, state, B, HK, HV, Dk, Dv, scale, qk_l2norm, gdn::DecodeOutGate{}, o, stream);
+}
+
+gdn_status gdn_decode_step_fused_outgate(const void* x, gdn_dtype io_dtype, const float* conv_w,
+                                         const float* conv_state_in, float* conv_state_out, int32_t conv_act,
+                                         const void* a, const void* b, gdn_dtype ab_dtype, const float* A_log,
+                                         const float* dt_bias, float* state, int32_t B, int32_t HK, int32_t HV,
+                                         int32_t Dk, int32_t Dv, float scale, int32_t qk_l2norm, const void* z,
+                                         const float* norm_w, float eps, void* o, void* stream) {
+    if (!z) return GDN_ERR_NULL;
+    return decode_fused_impl(x, io_dtype, conv_w, conv_state_in, conv_state_out, conv_act, a, b, ab_dtype, A_log,
+                             dt_bias, state, B, HK, HV, Dk, Dv, scale, qk_l2norm, gdn::DecodeOutGate{z, norm_w, eps},
+                             o, stream);
 }
 
 gdn_status gdn_conv_prefill(const void* x, gdn_dtype io_dtype, const float* conv_w, const float* conv_state_in,

@@ -99,9 +99,17 @@ struct DecodeConv {
     float* state_out;         // [B, 3, C]
     int act;                  // 0 identity, 1 SiLU
 };
+// The output epilogue of a decode step: out = o rsqrt(mean(o^2) + eps) (1 + w) sigmoid(z) over
+// each (sequence, value head) row of Dv values, before the store (z == nullptr: none).
+struct DecodeOutGate {
+    const void* z;            // [B, HV, Dv] io dtype
+    const float* w;           // [Dv]
+    float eps;
+};
 // Dk = Dv = 128 only.
 cudaError_t launch_decode_conv(bool bf16, const DecodeConv& conv, const DecodeGates& gates, float* state, int B,
-                               int HK, int HV, float scale, int l2norm, void* o, cudaStream_t s);
+                               int HK, int HV, float scale, int l2norm, void* o, const DecodeOutGate& og,
+                               cudaStream_t s);
 
 // Tiled tensor map (element strides 1, no interleave, zero fill out of range); false if the
 // driver entry point is missing or the encoder rejects the arguments.

@@ -321,6 +321,16 @@ class FusedDecodeSetup:
         b = self.base
         return 2 * b.HK * b.Dk + b.HV * b.Dv
 
+    def out_z(self, s: int) -> Tensor:
+        """Output-gate input of step ``s``: z [B, HV, Dv] ~ N(0, 1) in the io dtype."""
+        b = self.base
+        return _store(_rng(b.seed, 200, s, 9).standard_normal((b.B, b.HV, b.Dv), dtype=np.float32), b.io_dtype)
+
+    def out_w(self) -> np.ndarray:
+        """Output-norm weight w [Dv] ~ N(0, 0.3^2) fp32 (the recipe of outgate_inputs)."""
+        b = self.base
+        return (0.3 * _rng(b.seed, 200, 0, 10).standard_normal(b.Dv, dtype=np.float32)).astype(np.float32)
+
     def step(self, s: int):
         b = self.base
         x = _store(_rng(b.seed, 200, s, 1).standard_normal((b.B, self.C), dtype=np.float32), b.io_dtype)

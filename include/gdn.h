@@ -444,6 +444,30 @@ GDN_API gdn_status gdn_decode_step_fused(const void* x, gdn_dtype io_dtype,
                            float scale, int32_t qk_l2norm, void* o, void* stream);
 
 /*
+ * gdn_decode_step_fused_outgate -- gdn_decode_step_fused with the output epilogue applied to
+ * each output row before the store:
+ *     out = o * rsqrt(mean(o^2) + eps) * (1 + norm_w) * sigmoid(z)
+ * per (sequence, value head) over its Dv values: the zero-centred RMSNorm of the
+ * "Gated DeltaNet ... Qwen3-next" page (section 3.2: a norm weight initialised to zero, so
+ * stored as w with the scale 1 + w) and the sigmoid output gate of the GDN resource-
+ * allocation page; the same epilogue as gdn_chunk_prefill_outgate, so a sequence prefilled
+ * with that call continues here.  sigmoid is formed from the hardware tanh (absolute error
+ * below 2^-12).
+ *   z        [B, HV, Dv] io_dtype                                   (read)
+ *   norm_w   [Dv] fp32, eps >= 0                                    (read)
+ *   everything else as gdn_decode_step_fused (Dk = Dv = 128).
+ * Errors: those of gdn_decode_step_fused; NULL for z or norm_w NULL, SHAPE for eps < 0 or
+ * NaN, ALIGN, ALIAS also for the outputs over z or norm_w.
+ */
+GDN_API gdn_status gdn_decode_step_fused_outgate(const void* x, gdn_dtype io_dtype,
+                           const float* conv_w, const float* conv_state_in, float* conv_state_out,
+                           int32_t conv_act, const void* a, const void* b, gdn_dtype ab_dtype,
+                           const float* A_log, const float* dt_bias, float* state,
+                           int32_t B, int32_t HK, int32_t HV, int32_t Dk, int32_t Dv,
+                           float scale, int32_t qk_l2norm, const void* z, const float* norm_w,
+                           float eps, void* o, void* stream);
+
+/*
  * gdn_decode_status -- synchronises the current device and writes its decode error
  * word (GDN_DEVERR_NONE or GDN_DEVERR_TIMEOUT, shared by every decode launch on that
  * device) into *device_error, then clears it.  This is library bookkeeping with no

@@ -327,3 +327,23 @@ def test_prefill_gated_validation(L):
     assert call(ga=A + 192 * MB + 4) == 3      # misaligned
     assert call(o=A + 192 * MB) == 5           # output over a gate input
     assert call(ws_bytes=16) == 6
+
+
+def test_decode_fused_outgate_validation(L):
+    C = 2 * 2 * 128 + 4 * 128
+    def call(**kw):
+        a = dict(x=A, cw=A + 8 * MB, csi=A + 16 * MB, cso=A + 24 * MB, ga=A + 32 * MB, gb=A + 33 * MB,
+                 Al=A + 34 * MB, dtb=A + 35 * MB, st=A + 64 * MB, B=2, HK=2, HV=4, z=A + 40 * MB,
+                 nw=A + 41 * MB, eps=1e-6, o=A + 48 * MB)
+        a.update(kw)
+        return L.gdn_decode_step_fused_outgate(a["x"], 1, a["cw"], a["csi"], a["cso"], 1, a["ga"], a["gb"], 0,
+                                               a["Al"], a["dtb"], a["st"], a["B"], a["HK"], a["HV"], 128, 128,
+                                               1.0, 1, a["z"], a["nw"], a["eps"], a["o"], None)
+    assert call(z=None) == 1
+    assert call(nw=None) == 1
+    assert call(eps=-1.0) == 2
+    assert call(eps=float("nan")) == 2
+    assert call(z=A + 40 * MB + 8) == 3
+    assert call(o=A + 40 * MB) == 5      # output over z
+    assert call(st=A + 41 * MB) == 5     # state over norm_w
+    assert call(HV=3) == 2
