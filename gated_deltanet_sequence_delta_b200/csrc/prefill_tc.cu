@@ -54,6 +54,8 @@ constexpr int D = 128;     // head dim (Dk = Dv) of this path
 constexpr int NS = 32;     // value columns per carry CTA
 constexpr int NSTAGE = 2;  // TMA ring depth of the carry kernel
 constexpr int SC_FLOATS = 256;   // per (chunk, value head): a[64], d[64], scalars below
+constexpr int MS = 68;           // row stride (floats) of the chunk-local L / T buffer: rows
+                                 //   start on 16-byte boundaries for vector accesses
 constexpr int SC_GC = 128;       //   gamma_C = exp(G at the chunk's last token)
 constexpr int SC_UINV = 129;     //   U is stored as fp16(U * 2^-e); this holds 2^e
 constexpr int SC_VMAX = 130;     //   max |v| over the chunk's tile of this value head
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(1024) chunk_table_kernel(const int32_t* __rest
 }
 
 // ======================================================================================
-// In-place T = (I + L)^-1 for a 64 x 64 strictly lower L held in M (fp32, row stride 65),
+// In-place T = (I + L)^-1 for a 64 x 64 strictly lower L held in M (fp32, row stride MS),
 // 128 threads.  On return the strictly lower triangle of M holds T (its unit diagonal is
 // implied); entries on and above the diagonal are untouched.  Blocks of 16:
 //  * diagonal blocks T_bb = (I + L_bb)^-1 by right-looking column substitution: every
@@ -176,12 +178,12 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint
 // Element (r, c) of a 16 x 16 block of M at (r0, c0); UNIT: the block is a diagonal block
 // of T (unit diagonal implied, zero above it).
 template <bool UNIT>
-__device__ __forceinline__ float blk(const float (*M)[65], int r0, int c0, int r, int c) {
+__device__ __forceinline__ float blk(const float (*M)[MS], int r0, int c0, int r, int c) {
     if (UNIT) return r == c ? 1.f : (r > c ? M[r0 + r][c0 + c] : 0.f);
     return M[r0 + r][c0 + c];
 }
 template <bool UNIT>
-__device__ __forceinline__ void frag_a(uint32_t* a, const float (*M)[65], int r0, int c0, int g, int q) {
+__device__ __forceinline__ void frag_a(uint32_t* a, const float (*M)[MS], int r0, int c0, int g, int q) {
     a[0] = pack_h2(blk<UNIT>(M, r0, c0, g, 2 * q), blk<UNIT>(M, r0, c0, g, 2 * q + 1));
     a[1] = pack_h2(blk<UNIT>(M, r0, c0, g + 8, 2 * q), blk<UNIT>(M, r0, c0, g + 8, 2 * q + 1));
     a[2] = pack_h2(blk<UNIT>(M, r0, c0, g, 2 * q + 8), blk<UNIT>(M, r0, c0, g, 2 * q + 9));
@@ -189,14 +191,14 @@ __device__ __forceinline__ void frag_a(uint32_t* a, const float (*M)[65], int r0
 }
 // B fragment of the 16 x 8 slice (all 16 rows, columns n0 .. n0+7) of a block
 template <bool UNIT>
-__device__ __forceinline__ void frag_b(uint32_t* b, const float (*M)[65], int r0, int c0, int n0, int g, int q) {
+__device__ __forceinline__ void frag_b(uint32_t* b, const float (*M)[MS], int r0, int c0, int n0, int g, int q) {
     b[0] = pack_h2(blk<UNIT>(M, r0, c0, 2 * q, n0 + g), blk<UNIT>(M, r0, c0, 2 * q + 1, n0 + g));
     b[1] = pack_h2(blk<UNIT>(M, r0, c0, 2 * q + 8, n0 + g), blk<UNIT>(M, r0, c0, 2 * q + 9, n0 + g));
 }
 
 // Block row I of T: warp j (< I) forms X_j = sum_{k=j}^{I-1} L_Ik T_kj, then T_Ij = -T_II X_j.
 template <int I>
-__device__ __forceinline__ void tinv_row_block(float (*M)[65], float (*X)[16][17], int tid) {
+__device__ __forceinline__ void tinv_row_block(float (*M)[MS], float (*X)[16][17], int tid) {
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
     const float(*Xc)[17] = nullptr;
     if (warp < I) {
@@ -246,7 +248,7 @@ __device__ __forceinline__ void tinv_row_block(float (*M)[65], float (*X)[16][17
     __syncthreads();
 }
 
-__device__ __forceinline__ void tinv64_inplace(float (*M)[65], float (*X)[16][17], int tid) {
+__device__ __forceinline__ void tinv64_inplace(float (*M)[MS], float (*X)[16][17], int tid) {
     float col[16];
     const int b = tid >> 4, c = tid & 15, o = 16 * b;
     if (tid < 64) {
@@ -279,18 +281,20 @@ struct PrepSmem {
     // rewritten in place as fp16 K_hat; rows 64-127 are reused for V (bf16 from TMA, then
     // fp16 V * sv in place) once Q_hat has been written out.
     uint16_t KQ[2][128 * 64];
-    // L, then T in place (fp32, row stride 65); then, in the same bytes, the fp16 MMA
+    // L, then T in place (fp32, row stride MS); then, in the same bytes, the fp16 MMA
     // operands T diag(b gamma) (bytes 0-8191) and T diag(b) (8192-16383), K-major 128B-swizzled
-    float M[64][65];
+    float M[64][MS];
     float X[3][16][17];
     float rk[64], rq[64], G[64], bt[64], bgr[64], red[8];
-    float eu[64];   // rk_j exp(G_r - G_j), the token factor of the separated decays
+    alignas(16) float eu[64];   // rk_j exp(G_r - G_j), the token factor of the separated decays
     float ga[2][64], ba[2][64];   // g, beta of value head gi in slot gi % 2, loaded ahead
     uint64_t bar_load, bar_v, bar_mma;
     uint32_t tmem_base;
+    uint32_t nv;   // V tile copies issued so far (thread 96)
 };
 static_assert(offsetof(PrepSmem, M) % 1024 == 0, "the swizzled operands in M need 1024-byte alignment");
 constexpr size_t kPrepSmemBytes = sizeof(PrepSmem) + 1024;
+static_assert(4 * (kPrepSmemBytes + 1024) <= 228 * 1024, "four chunk_prep CTAs per SM (1 KB reserved each)");
 constexpr uint32_t kPrepTmemCols = 128;   // 4 resident CTAs fill the 512 columns
 
 // Column t = tid of a 64 x 128 fp16 tile from TMEM lane t (64 fp32 columns = the tile's 64
@@ -320,8 +324,9 @@ __global__ void __launch_bounds__(128, 4)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const DecodeGates gs, const int32_t* __restrict__ cu,
                   const int32_t* __restrict__ chunk_off, int64_t T, int n_seqs, int HV, float scale,
-                  int l2norm, int HK, f16* __restrict__ Wg, f16* __restrict__ Ug, f16* __restrict__ Pg,
-                  f16* __restrict__ QKg, float* __restrict__ SCg, int32_t* __restrict__ status, int stall) {
+                  int l2norm, int HK, f16* __restrict__ Wg, f16* __restrict__ Ug,
+                  const __grid_constant__ CUtensorMap tm_p_st, const __grid_constant__ CUtensorMap tm_qk_st,
+                  float* __restrict__ SCg, int32_t* __restrict__ status, int stall) {
     extern __shared__ uint8_t smem_raw[];
     PrepSmem& S = *reinterpret_cast<PrepSmem*>(align1024(smem_raw));
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -340,6 +345,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc::mbar_init(&S.bar_v, 1);
         tc::mbar_init(&S.bar_mma, 1);
         tc::fence_mbar_init();
+        S.nv = 0;
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -353,7 +359,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int si = (int)s;
     uint8_t* kq = reinterpret_cast<uint8_t*>(&S.KQ[0][0]);
     uint32_t mma_phase = 0;
-    int v_loads = 0;   // V tile copies issued (thread 0)
 
     if (tid == 0) {
         tc::mbar_expect_tx(&S.bar_load, 4 * 64 * 64 * 2);
@@ -414,10 +419,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     {
         const float rki = tid < 64 ? S.rk[tid] : 0.f;
         const float rqi = tid >= 64 ? S.rq[tid - 64] : 0.f;
-        {   // K_hat (tid < 64) / Q_hat row: fp16 in place (K_hat feeds the W MMA) and out to
-            // global in natural column order; rows past the chunk are zeroed
+        {   // K_hat (tid < 64) / Q_hat row: fp16 in place (K_hat feeds the W MMA, and both go
+            // out from there by tensor-map stores); rows past the chunk are zeroed
             const float rr = tid < cn || (tid >= 64 && tid - 64 < cn) ? (tid < 64 ? rki : rqi) : 0.f;
-            uint4* dst = reinterpret_cast<uint4*>(QKg + (((size_t)chunk * HK + hk) * 128 + tid) * D);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint4* row = reinterpret_cast<uint4*>(kq + half * 16384 + tid * 128);
@@ -429,27 +433,29 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     __align__(16) f16 hx[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) hx[t] = __float2half_rn(__bfloat162float(e[t]) * rr);
-                    const uint4 hv = *reinterpret_cast<const uint4*>(hx);
-                    row[pc] = hv;
-                    dst[half * 8 + c16] = hv;
+                    row[pc] = *reinterpret_cast<const uint4*>(hx);
                 }
             }
         }
         tc::fence_async_smem();
         __syncthreads();
-        // Q is consumed: its rows now receive V of the first value head (test hook,
-        // gdn_testing_stall: not for the first CTA, whose wait for it then runs out)
-        if (tid == 0 && !(stall && chunk == 0 && hk == 0)) {
-            tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
-            ++v_loads;
-            tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, hk * G, si);
-            tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, hk * G, si);
+        if (tid == 0) {   // [K_hat; Q_hat] of the (chunk, q/k head), 128 rows
+            const int qkrow = (chunk * HK + hk) * 128;
+            tc::tma_store_2d(&tm_qk_st, kq, 0, qkrow);
+            tc::tma_store_2d(&tm_qk_st, kq + 16384, 64, qkrow);
+            tc::tma_store_2d(&tm_qk_st, kq + 8192, 0, qkrow + 64);
+            tc::tma_store_2d(&tm_qk_st, kq + 16384 + 8192, 64, qkrow + 64);
+            tc::bulk_commit();
         }
+        // From here the Q rows of the first half stage each value head's P (written by
+        // threads 64-127, stored by thread 96), then take that head's V tile; the second
+        // half's Q rows take the rest of V.
 
         for (int gi = 0; gi < G; ++gi) {
             const int h = hk * G + gi;
             const size_t ch = (size_t)chunk * HV + h;
             const bool last = gi == G - 1;
+            if (gi == 0 && tid == 0) tc::bulk_wait_read<0>();   // Q_hat has left the staging rows
             // ---- running sum of the log-decays, write strengths -------------------------
             if (tid < 64) {
                 float gv = S.ga[gi & 1][tid];
@@ -489,8 +495,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const float Gi = S.G[i], bi = S.bt[i] * rki;
                     if (sep) {
                         const float ai = i < cn ? bi * __expf(Gi - Gr) : 0.f;
+                        float4* mrow = reinterpret_cast<float4*>(&S.M[i][0]);
+                        const float4* eu4 = reinterpret_cast<const float4*>(S.eu);
 #pragma unroll
-                        for (int j = 0; j < 64; ++j) S.M[i][j] = j < i ? ai * S.eu[j] * row[j] : 0.f;
+                        for (int j4 = 0; j4 < 16; ++j4) {
+                            const float4 e = eu4[j4];
+                            const int j = 4 * j4;
+                            float4 l;
+                            l.x = j < i ? ai * e.x * row[j] : 0.f;
+                            l.y = j + 1 < i ? ai * e.y * row[j + 1] : 0.f;
+                            l.z = j + 2 < i ? ai * e.z * row[j + 2] : 0.f;
+                            l.w = j + 3 < i ? ai * e.w * row[j + 3] : 0.f;
+                            mrow[j4] = l;
+                        }
                     } else {
 #pragma unroll
                         for (int j = 0; j < 64; ++j) {
@@ -505,34 +522,58 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const float Gi = S.G[i], qi = scale * rqi;
                     SCg[ch * SC_FLOATS + i] = i < cn ? scale * expf(Gi) : 0.f;
                     if (i == 0) SCg[ch * SC_FLOATS + SC_GC] = expf(Gl);
-                    uint4* prow = reinterpret_cast<uint4*>(Pg + (ch * 64 + i) * 64);
+                    uint8_t* prow = kq + 8192 + i * 128;   // 128B-swizzled like the tensor map
                     const float ai = sep && i < cn ? qi * __expf(Gi - Gr) : 0.f;
+                    const float4* eu4 = reinterpret_cast<const float4*>(S.eu);
 #pragma unroll
                     for (int c8 = 0; c8 < 8; ++c8) {
                         __align__(16) f16 e[8];
+                        const float4 ea = eu4[2 * c8], eb = eu4[2 * c8 + 1];
+                        const float ev[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
 #pragma unroll
                         for (int t = 0; t < 8; ++t) {
                             const int j = c8 * 8 + t;
                             float v = 0.f;
-                            if (sep) v = j <= i ? ai * S.eu[j] * row[j] : 0.f;
+                            if (sep) v = j <= i ? ai * ev[t] * row[j] : 0.f;
                             else if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
                             e[t] = __float2half_rn(v);
                         }
-                        prow[c8] = *reinterpret_cast<const uint4*>(e);
+                        *reinterpret_cast<uint4*>(prow + ((c8 ^ (i & 7)) << 4)) = *reinterpret_cast<const uint4*>(e);
                     }
                 }
             }
+            tc::fence_async_smem();
             __syncthreads();
+            if (tid == 96) {
+                // warp 3 has no part in the inverse's first phase: P out, then this head's V
+                // into the staging rows once the store has read them (test hook,
+                // gdn_testing_stall: no V for the first CTA's first head, whose wait then runs out)
+                tc::tma_store_2d(&tm_p_st, kq + 8192, 0, (int)(ch * 64));
+                tc::bulk_commit();
+                tc::bulk_wait_read<0>();
+                if (!(stall && chunk == 0 && hk == 0 && gi == 0)) {
+                    tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
+                    ++S.nv;
+                    tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, h, si);
+                    tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, h, si);
+                }
+            }
             tinv64_inplace(S.M, S.X, tid);
             // ---- fp16 MMA operands T diag(b gamma) and T diag(b), 128B-swizzled, written
             //      over M once every thread holds its part of T -----------------------------
             {
                 const int i = tid >> 1, c0 = (tid & 1) * 32;
                 float tv[32];
+                const float4* mrow = reinterpret_cast<const float4*>(&S.M[i][c0]);
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const int j = c0 + t;
-                    tv[t] = j < i ? S.M[i][j] : (j == i ? 1.f : 0.f);
+                for (int t4 = 0; t4 < 8; ++t4) {
+                    const float4 m4 = mrow[t4];
+                    const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = c0 + 4 * t4 + e;
+                        tv[4 * t4 + e] = j < i ? mv[e] : (j == i ? 1.f : 0.f);
+                    }
                 }
                 __syncthreads();
                 uint8_t* aw = reinterpret_cast<uint8_t*>(&S.M[0][0]);
@@ -631,29 +672,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mma_phase ^= 1;
                 if (__syncthreads_or(!ok)) goto abort;
                 tc::tc_fence_after();
-                if (tid == 0) {   // the V rows are free again: next head's V
-                    tc::mbar_expect_tx(&S.bar_v, 2 * 64 * 64 * 2);
-                    ++v_loads;
-                    tc::tma_load_3d(kq + 8192, &tm_v, &S.bar_v, 0, h + 1, si);
-                    tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, h + 1, si);
-                }
             }
             store_tile_from_tmem(Ug + ch * 64 * D, (last ? tG : tW) + lane_base, tid);
             tc::tc_fence_before();
             __syncthreads();   // TMEM reads done; M (the operands) free for the next head
         }
     }
+    if (tid == 0 || tid == 96) tc::bulk_wait<0>();   // this thread's tensor-map stores are done
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kPrepTmemCols);
     return;
 abort:
+    if (tid == 0 || tid == 96) tc::bulk_wait<0>();
     if (tid == 0) {
         record_timeout(status);
         // the copies and products still in flight land before the shared memory and TMEM are
         // released; each wait is for the latest phase of its barrier (at once if complete)
         (void)tc::mbar_wait(&S.bar_load, 0, 50000000ull);
-        if (v_loads > 0) (void)tc::mbar_wait(&S.bar_v, (uint32_t)((v_loads - 1) & 1), 50000000ull);
+        const uint32_t nv = S.nv;
+        if (nv > 0) (void)tc::mbar_wait(&S.bar_v, (nv - 1u) & 1u, 50000000ull);
         (void)tc::mbar_wait(&S.bar_mma, mma_phase ^ 1u, 50000000ull);
     }
     tc::tc_fence_before();
@@ -1285,7 +1323,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, void* workspace, cudaStream_
                                            (int)cudaSharedmemCarveoutMaxShared);
             if (err != cudaSuccess) return err;
             kern<<<grid, 128, kPrepSmemBytes, s>>>(tq, tk, tv, a.gates, a.cu, chunk_off, a.T, a.n_seqs, a.HV,
-                                                   a.scale, a.l2norm, a.HK, W, U, P, QK, SC, a.status,
+                                                   a.scale, a.l2norm, a.HK, W, U, tp, tqk, SC, a.status,
                                                    testing_stall_site() == GDN_STALL_PREFILL_PREP ? 1 : 0);
             return cudaSuccess;
         };
