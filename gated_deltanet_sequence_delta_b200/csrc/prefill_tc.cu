@@ -719,7 +719,8 @@ struct CarrySmem {
                            //   by chunk parity
     f16 Dl[C * NS];        // scaled Delta, same layout (K = tokens)
     f16 Dt[C * NS];        // scaled Delta~ = diag(exp(G_C - G)) Delta
-    ZSlot zr[NZ];          // output epilogue: z tiles and scalars, chunk c in slot c % NZ
+    alignas(128) ZSlot zr[NZ];   // output epilogue: z tiles and scalars, chunk c in slot c % NZ
+                                 //   (tensor-map copy targets: 128-byte aligned)
     float red[4];
     // output epilogue: per chunk parity, this CTA's per-row sums of squares and those
     // received from the other slices (bulk-copy source and target: 16-byte aligned)
@@ -740,7 +741,7 @@ static_assert(sizeof(CarryStage) % 1024 == 0 && offsetof(CarryStage, K) % 1024 =
                   offsetof(CarryStage, P) % 1024 == 0 && offsetof(CarryStage, U) % 16 == 0 &&
                   offsetof(CarryStage, SC) % 16 == 0,
               "carry stage layout");
-static_assert(offsetof(CarrySmem, zr) % 16 == 0 && sizeof(ZSlot) % 16 == 0 && offsetof(ZSlot, a) % 16 == 0 &&
+static_assert(offsetof(CarrySmem, zr) % 128 == 0 && sizeof(ZSlot) % 128 == 0 && offsetof(ZSlot, a) % 16 == 0 &&
                   offsetof(CarrySmem, oloc) % 16 == 0 && offsetof(CarrySmem, opart) % 16 == 0 &&
                   offsetof(CarrySmem, H0) % 16 == 0 && offsetof(CarrySmem, Dl) % 16 == 0 &&
                   offsetof(CarrySmem, Dt) % 16 == 0,
