@@ -429,11 +429,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int c16 = 0; c16 < 8; ++c16) {
                     const int pc = c16 ^ (tid & 7);   // logical chunk c16 sits at c16 ^ (row % 8)
                     const uint4 u = row[pc];
-                    const bf16* e = reinterpret_cast<const bf16*>(&u);
-                    __align__(16) f16 hx[8];
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t hv[4];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) hx[t] = __float2half_rn(__bfloat162float(e[t]) * rr);
-                    row[pc] = *reinterpret_cast<const uint4*>(hx);
+                    for (int q = 0; q < 4; ++q) {   // bf16 pair -> two floats (exact) -> fp16 pair
+                        const __half2 h2 = __floats2half2_rn(__uint_as_float(w[q] << 16) * rr,
+                                                             __uint_as_float(w[q] & 0xffff0000u) * rr);
+                        hv[q] = *reinterpret_cast<const uint32_t*>(&h2);
+                    }
+                    row[pc] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
                 }
             }
         }
@@ -530,14 +534,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         __align__(16) f16 e[8];
                         const float4 ea = eu4[2 * c8], eb = eu4[2 * c8 + 1];
                         const float ev[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
+                        float pv[8];
 #pragma unroll
                         for (int t = 0; t < 8; ++t) {
                             const int j = c8 * 8 + t;
                             float v = 0.f;
                             if (sep) v = j <= i ? ai * ev[t] * row[j] : 0.f;
                             else if (j <= i && i < cn) v = qi * __expf(Gi - S.G[j]) * S.rk[j] * row[j];
-                            e[t] = __float2half_rn(v);
+                            pv[t] = v;
                         }
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) reinterpret_cast<__half2*>(e)[t] = __floats2half2_rn(pv[2 * t], pv[2 * t + 1]);
                         *reinterpret_cast<uint4*>(prow + ((c8 ^ (i & 7)) << 4)) = *reinterpret_cast<const uint4*>(e);
                     }
                 }
@@ -599,31 +606,38 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             {
                 const int r = tid >> 1, half = tid & 1;
                 uint4* vr = reinterpret_cast<uint4*>(kq + half * 16384 + 8192 + r * 128);
-                float vmax = 0.f;
+                // max |v| from the bf16 bit patterns: with the sign bit cleared, their order as
+                // 16-bit integers is the order of the magnitudes (a NaN pattern exceeds them all
+                // and turns the scale off, as an infinite value does)
+                uint32_t m2 = 0;
                 if (r < cn) {
 #pragma unroll
                     for (int c16 = 0; c16 < 8; ++c16) {
                         const uint4 u = vr[c16 ^ (r & 7)];
-                        const bf16* e = reinterpret_cast<const bf16*>(&u);
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) vmax = fmaxf(vmax, fabsf(__bfloat162float(e[t])));
+                        m2 = __vmaxu2(m2, u.x & 0x7fff7fffu);
+                        m2 = __vmaxu2(m2, u.y & 0x7fff7fffu);
+                        m2 = __vmaxu2(m2, u.z & 0x7fff7fffu);
+                        m2 = __vmaxu2(m2, u.w & 0x7fff7fffu);
                     }
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-                if ((tid & 31) == 0) S.red[warp] = vmax;
+                const uint32_t mw = __reduce_max_sync(0xffffffffu, max(m2 & 0xffffu, m2 >> 16));
+                if ((tid & 31) == 0) S.red[warp] = __uint_as_float(mw << 16);
                 __syncthreads();
-                vmax = fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3]));
+                const float vmax = fmaxf(fmaxf(S.red[0], S.red[1]), fmaxf(S.red[2], S.red[3]));
                 const float uinv = pow2_above(vmax), sv = r < cn ? 1.f / uinv : 0.f;
 #pragma unroll
-                for (int c16 = 0; c16 < 8; ++c16) {
+                for (int c16 = 0; c16 < 8; ++c16) {   // bf16 pair -> two floats (exact) -> fp16 pair
                     const int pc = c16 ^ (r & 7);
                     const uint4 u = vr[pc];
-                    const bf16* e = reinterpret_cast<const bf16*>(&u);
-                    __align__(16) f16 hx[8];
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t hv[4];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) hx[t] = __float2half_rn(__bfloat162float(e[t]) * sv);
-                    vr[pc] = *reinterpret_cast<const uint4*>(hx);
+                    for (int q = 0; q < 4; ++q) {
+                        const __half2 h2 = __floats2half2_rn(__uint_as_float(w[q] << 16) * sv,
+                                                             __uint_as_float(w[q] & 0xffff0000u) * sv);
+                        hv[q] = *reinterpret_cast<const uint32_t*>(&h2);
+                    }
+                    vr[pc] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
                 }
                 if (tid == 0) {
                     SCg[ch * SC_FLOATS + SC_UINV] = uinv;
