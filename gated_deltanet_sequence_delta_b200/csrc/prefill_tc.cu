@@ -152,13 +152,18 @@ __global__ void __launch_bounds__(1024) chunk_table_kernel(const int32_t* __rest
 // ======================================================================================
 // In-place T = (I + L)^-1 for a 64 x 64 strictly lower L held in M (fp32, row stride MS),
 // 128 threads.  On return the strictly lower triangle of M holds T (its unit diagonal is
-// implied); entries on and above the diagonal are untouched.  Blocks of 16:
-//  * diagonal blocks T_bb = (I + L_bb)^-1 by right-looking column substitution: every
-//    finished x_j updates all later rows at once, so the dependent chain is one FMA per row;
-//  * block rows I = 1, 2, 3: T_Ij = -T_II sum_{k=j}^{I-1} L_Ik T_kj for all j < I at once,
-//    one warp per j, the 16 x 16 block products on mma.sync with fp16 operands (the T
-//    entries are rounded to fp16 for the W / U operands anyway).  Row block I of L is
-//    read only while row block I of T is formed, so T overwrites it.
+// implied); entries on and above the diagonal are untouched.  With 16 x 16 blocks (b, b')
+// and the 32 x 32 halves A (blocks 0, 1) and B (blocks 2, 3):
+//  * the four diagonal blocks T_bb = (I + L_bb)^-1 by right-looking column substitution
+//    (one thread per column; every finished x_j updates all later rows at once, so the
+//    dependent chain is one FMA per row);
+//  * inside each half, T_10 = -T_11 L_10 T_00 and T_32 = -T_33 L_32 T_22, one warp each;
+//  * the lower-left half T_BA = -T_B (L_BA T_A): first the four blocks of Y = L_BA T_A, then
+//    the four of -T_B Y, one warp per block.
+// The block products run on mma.sync with fp16 operands and fp32 accumulation (the T
+// entries are rounded to fp16 for the W / U operands anyway); the intermediate products go
+// through shared memory as fp16, transposed so that a B fragment is one 32-bit load.  Five
+// CTA barriers.
 // ======================================================================================
 // Warp-level 16x16x16 products on the legacy tensor-core path (mma.sync m16n8k16, fp16
 // operands, fp32 accumulation); fragment layouts of that instruction: g = lane / 4,
@@ -196,81 +201,111 @@ __device__ __forceinline__ void frag_b(uint32_t* b, const float (*M)[MS], int r0
     b[1] = pack_h2(blk<UNIT>(M, r0, c0, 2 * q + 8, n0 + g), blk<UNIT>(M, r0, c0, 2 * q + 9, n0 + g));
 }
 
-// Block row I of T: warp j (< I) forms X_j = sum_{k=j}^{I-1} L_Ik T_kj, then T_Ij = -T_II X_j.
-template <int I>
-__device__ __forceinline__ void tinv_row_block(float (*M)[MS], float (*X)[16][17], int tid) {
-    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-    const float(*Xc)[17] = nullptr;
-    if (warp < I) {
-        const int j = warp;
-        float acc[2][4] = {};
+// B fragment (rows 2q, 2q+1, 2q+8, 2q+9 of column n0 + g) of a 16 x 16 block held
+// transposed in fp16 (Yt[n][k] = Y[k][n])
+__device__ __forceinline__ void frag_b_t(uint32_t* b, const __half (*Yt)[18], int n0, int g, int q) {
+    b[0] = *reinterpret_cast<const uint32_t*>(&Yt[n0 + g][2 * q]);
+    b[1] = *reinterpret_cast<const uint32_t*>(&Yt[n0 + g][2 * q + 8]);
+}
+// a 16 x 16 product (the accumulators of two 16 x 8 tiles), transposed, as fp16
+__device__ __forceinline__ void store_d_t(__half (*Yt)[18], const float (*acc)[4], int g, int q) {
 #pragma unroll
-        for (int k = 0; k < I; ++k) {
-            if (k < j) continue;
-            uint32_t a[4], b[2];
-            frag_a<false>(a, M, 16 * I, 16 * k, g, q);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                if (k == j) frag_b<true>(b, M, 16 * k, 16 * j, 8 * nt, g, q);
-                else frag_b<false>(b, M, 16 * k, 16 * j, 8 * nt, g, q);
-                mma16816(acc[nt], a, b);
-            }
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            X[j][g][8 * nt + 2 * q] = acc[nt][0];
-            X[j][g][8 * nt + 2 * q + 1] = acc[nt][1];
-            X[j][g + 8][8 * nt + 2 * q] = acc[nt][2];
-            X[j][g + 8][8 * nt + 2 * q + 1] = acc[nt][3];
-        }
+    for (int nt = 0; nt < 2; ++nt) {
+        Yt[8 * nt + 2 * q][g] = __float2half_rn(acc[nt][0]);
+        Yt[8 * nt + 2 * q + 1][g] = __float2half_rn(acc[nt][1]);
+        Yt[8 * nt + 2 * q][g + 8] = __float2half_rn(acc[nt][2]);
+        Yt[8 * nt + 2 * q + 1][g + 8] = __float2half_rn(acc[nt][3]);
     }
-    __syncthreads();   // every read of row block I of L is done before it is overwritten
-    if (warp < I) {
-        const int j = warp;
-        Xc = X[j];
-        float acc[2][4] = {};
-        uint32_t a[4], b[2];
-        frag_a<true>(a, M, 16 * I, 16 * I, g, q);
+}
+// -(a 16 x 16 product) into block (bi, bj) of M
+__device__ __forceinline__ void store_neg_block(float (*M)[MS], const float (*acc)[4], int bi, int bj, int g, int q) {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            b[0] = pack_h2(Xc[2 * q][8 * nt + g], Xc[2 * q + 1][8 * nt + g]);
-            b[1] = pack_h2(Xc[2 * q + 8][8 * nt + g], Xc[2 * q + 9][8 * nt + g]);
-            mma16816(acc[nt], a, b);
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            M[16 * I + g][16 * j + 8 * nt + 2 * q] = -acc[nt][0];
-            M[16 * I + g][16 * j + 8 * nt + 2 * q + 1] = -acc[nt][1];
-            M[16 * I + g + 8][16 * j + 8 * nt + 2 * q] = -acc[nt][2];
-            M[16 * I + g + 8][16 * j + 8 * nt + 2 * q + 1] = -acc[nt][3];
-        }
+    for (int nt = 0; nt < 2; ++nt) {
+        M[16 * bi + g][16 * bj + 8 * nt + 2 * q] = -acc[nt][0];
+        M[16 * bi + g][16 * bj + 8 * nt + 2 * q + 1] = -acc[nt][1];
+        M[16 * bi + g + 8][16 * bj + 8 * nt + 2 * q] = -acc[nt][2];
+        M[16 * bi + g + 8][16 * bj + 8 * nt + 2 * q + 1] = -acc[nt][3];
     }
-    __syncthreads();
 }
 
-__device__ __forceinline__ void tinv64_inplace(float (*M)[MS], float (*X)[16][17], int tid) {
-    float col[16];
-    const int b = tid >> 4, c = tid & 15, o = 16 * b;
-    if (tid < 64) {
+__device__ __forceinline__ void tinv64_inplace(float (*M)[MS], __half (*Y)[16][18], int tid) {
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+    {   // ---- diagonal blocks -----------------------------------------------------------
+        float col[16];
+        const int b = tid >> 4, c = tid & 15, o = 16 * b;
+        if (tid < 64) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) col[i] = (i == c) ? 1.f : 0.f;
+            for (int i = 0; i < 16; ++i) col[i] = (i == c) ? 1.f : 0.f;
 #pragma unroll
-        for (int j = 0; j < 15; ++j) {
-            const float xj = col[j];
+            for (int j = 0; j < 15; ++j) {
+                const float xj = col[j];
 #pragma unroll
-            for (int i = j + 1; i < 16; ++i) col[i] = fmaf(-M[o + i][o + j], xj, col[i]);
+                for (int i = j + 1; i < 16; ++i) col[i] = fmaf(-M[o + i][o + j], xj, col[i]);
+            }
         }
-    }
-    __syncthreads();   // all reads of the diagonal blocks of L precede their overwrite
-    if (tid < 64) {
+        __syncthreads();   // all reads of the diagonal blocks of L precede their overwrite
+        if (tid < 64) {
 #pragma unroll
-        for (int i = 1; i < 16; ++i)
-            if (i > c) M[o + i][o + c] = col[i];
+            for (int i = 1; i < 16; ++i)
+                if (i > c) M[o + i][o + c] = col[i];
+        }
+        __syncthreads();
+    }
+    uint32_t a[4], bb[2];
+    if (warp < 2) {   // ---- T_10 (warp 0) and T_32 (warp 1): -T_ii (L_ij T_jj) ------------------
+        const int i = 2 * warp + 1, j = i - 1;
+        float acc[2][4] = {};
+        frag_a<false>(a, M, 16 * i, 16 * j, g, q);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            frag_b<true>(bb, M, 16 * j, 16 * j, 8 * nt, g, q);
+            mma16816(acc[nt], a, bb);
+        }
+        store_d_t(Y[warp], acc, g, q);
+        __syncwarp();
+        float acc2[2][4] = {};
+        frag_a<true>(a, M, 16 * i, 16 * i, g, q);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            frag_b_t(bb, Y[warp], 8 * nt, g, q);
+            mma16816(acc2[nt], a, bb);
+        }
+        store_neg_block(M, acc2, i, j, g, q);
     }
     __syncthreads();
-    tinv_row_block<1>(M, X, tid);
-    tinv_row_block<2>(M, X, tid);
-    tinv_row_block<3>(M, X, tid);
+    const int bi = 2 + (warp >> 1), bj = warp & 1;   // this warp's block of the lower-left half
+    {   // ---- Y_ij = sum_{m >= j} L_im T_mj (T_A is lower) ----------------------------------
+        float acc[2][4] = {};
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            if (m < bj) continue;
+            frag_a<false>(a, M, 16 * bi, 16 * m, g, q);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                if (m == bj) frag_b<true>(bb, M, 16 * m, 16 * bj, 8 * nt, g, q);
+                else frag_b<false>(bb, M, 16 * m, 16 * bj, 8 * nt, g, q);
+                mma16816(acc[nt], a, bb);
+            }
+        }
+        store_d_t(Y[warp], acc, g, q);
+    }
+    __syncthreads();   // Y complete, and every read of L_BA done before T_BA overwrites it
+    {   // ---- T_ij = -sum_{k <= i} T_ik Y_kj (T_B is lower) -----------------------------------
+        float acc[2][4] = {};
+#pragma unroll
+        for (int k = 2; k < 4; ++k) {
+            if (k > bi) continue;
+            if (k == bi) frag_a<true>(a, M, 16 * bi, 16 * bi, g, q);
+            else frag_a<false>(a, M, 16 * bi, 16 * k, g, q);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                frag_b_t(bb, Y[(k - 2) * 2 + bj], 8 * nt, g, q);
+                mma16816(acc[nt], a, bb);
+            }
+        }
+        store_neg_block(M, acc, bi, bj, g, q);
+    }
+    __syncthreads();
 }
 
 // ======================================================================================
@@ -284,7 +319,7 @@ struct PrepSmem {
     // L, then T in place (fp32, row stride MS); then, in the same bytes, the fp16 MMA
     // operands T diag(b gamma) (bytes 0-8191) and T diag(b) (8192-16383), K-major 128B-swizzled
     float M[64][MS];
-    float X[3][16][17];
+    __half Y[4][16][18];   // the inverse's intermediate 16 x 16 products, transposed, fp16
     float rk[64], rq[64], G[64], bt[64], bgr[64], red[8];
     alignas(16) float eu[64];   // rk_j exp(G_r - G_j), the token factor of the separated decays
     float ga[2][64], ba[2][64];   // g, beta of value head gi in slot gi % 2, loaded ahead
@@ -565,7 +600,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tc::tma_load_3d(kq + 16384 + 8192, &tm_v, &S.bar_v, 64, h, si);
                 }
             }
-            tinv64_inplace(S.M, S.X, tid);
+            tinv64_inplace(S.M, S.Y, tid);
             // ---- fp16 MMA operands T diag(b gamma) and T diag(b), 128B-swizzled, written
             //      over M once every thread holds its part of T -----------------------------
             {
