@@ -330,6 +330,7 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
         }
         float4 hv[8];
         float pu[CPL] = {}, pq[CPL] = {};
+        float o_keep = 0.f;   // OUTG: this thread's output value, kept for the epilogue
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr) {
             const int row = warp * 8 + rr;
@@ -365,15 +366,8 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
             const float delta = bt * (ld_raw<QT>(B.v, j) - alpha * su * rk);
             const float oj = scale * (alpha * (sq * rq) + delta * kq);
             S.delta[j] = delta;
-            if (!OUTG) {
-                store_elem(o, (int64_t)bh * kSD + j, oj);
-            } else {   // the row's mean square over its 128 values: these four warps, one barrier
-                const float ss = warp_sum(oj * oj);
-                if (lane == 0) S.osq[warp] = ss;
-                tc::named_bar(2, kSD);
-                const float ms = (S.osq[0] + S.osq[1] + S.osq[2] + S.osq[3]) * (1.f / kSD);
-                store_elem(o, (int64_t)bh * kSD + j, oj * rsqrtf(ms + og.eps) * wj * sigmoid_tanh(zj));
-            }
+            if (!OUTG) store_elem(o, (int64_t)bh * kSD + j, oj);
+            else o_keep = oj;   // the output epilogue runs after the state update is under way
         }
         tc::named_bar(1, kSWarps * 32);
         // H' = alpha H + k_hat delta^T, written back in place
@@ -398,6 +392,17 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
             tc::bulk_commit();
             tc::bulk_wait_read<1>();   // the previous slice's store has read its slot
             if (i > 0) tc::mbar_arrive(&S.empty[(i - 1) % kSStages]);
+        }
+        if (OUTG && tid < kSD) {
+            // the output epilogue, behind the state update and its store: the row's mean square
+            // over its 128 values from these four warps (one barrier among them), then the
+            // norm, (1 + w) and the gate.  osq is rewritten only after the next item's CTA-wide
+            // barrier, which every reader here has passed first.
+            const float ss = warp_sum(o_keep * o_keep);
+            if (lane == 0) S.osq[warp] = ss;
+            tc::named_bar(2, kSD);
+            const float ms = (S.osq[0] + S.osq[1] + S.osq[2] + S.osq[3]) * (1.f / kSD);
+            store_elem(o, (int64_t)bh * kSD + tid, o_keep * rsqrtf(ms + og.eps) * wj * sigmoid_tanh(zj));
         }
     }
     if (tid == 0) tc::bulk_wait<0>();   // every store complete before the CTA exits
