@@ -226,6 +226,13 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
         tc::fence_mbar_init();
     }
     __syncthreads();
+    // Launched with programmatic stream serialisation: this grid may start while the kernel
+    // before it in the stream is still running.  Nothing in global memory is touched before
+    // that kernel has completed and its writes are visible; then the next grid may launch, its
+    // CTAs taking each SM as this grid's CTA there exits (every CTA of this grid is resident
+    // by then, so a waiting CTA of the next grid never holds an SM this grid still needs).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == kSWarps) {
         // ---------------- producer ----------------------------------------------------
@@ -435,10 +442,20 @@ cudaError_t launch_decode_staged(const void* q, const void* k, const void* v, co
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = n_items < sms ? n_items : sms;
-    decode_staged_kernel<IO, CONV, OUTG><<<grid, kSThreads, smem, s>>>(
-        (const IO*)q, (const IO*)k, (const IO*)v, conv, gates, state, n_items, HK, HV, scale, l2norm, (IO*)o,
-        testing_stall_site() == GDN_STALL_DECODE ? 1 : 0, og);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kSThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddepcontrol in the kernel
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_staged_kernel<IO, CONV, OUTG>, (const IO*)q, (const IO*)k, (const IO*)v, conv,
+                           gates, state, n_items, HK, HV, scale, l2norm, (IO*)o,
+                           testing_stall_site() == GDN_STALL_DECODE ? 1 : 0, og);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
 }

@@ -127,14 +127,16 @@ def test_conv_long_workload_sampled():
     assert cs.shape == (1, 3, C)
 
 
-def test_conv_prefill_decode_end_to_end():
+def _end_to_end(outgate):
     """Three packed sequences (37, 130, 64 tokens) from raw projections: the convolution,
     the chunked prefill from a carried state, then two fused decode steps that take over
     both states; against the oracle's convolution, gates and recurrence over the whole
     sequences (prefill tokens followed by the two decoded tokens).  gdn_conv_prefill hands
     the prefill q, k, v in the io dtype, so the oracle rounds the prefill tokens'
     convolution output to bf16 at the same point; the fused decode step keeps its q, k, v
-    in fp32, and so does the oracle for the decoded tokens."""
+    in fp32, and so does the oracle for the decoded tokens.  outgate: the output epilogue on
+    both calls (gdn_chunk_prefill_outgate, then the decode step's), against the oracle's
+    epilogue over the whole sequences."""
     import oracle
     import torch
     import gated_deltanet_sequence_delta_b200 as G
@@ -149,6 +151,10 @@ def test_conv_prefill_decode_end_to_end():
     b = rng.standard_normal((n_pre + 2 * N, HV)).astype(np.float32)
     A_log, dt_bias, _ = I.gate_params(87, HV)
     h0 = (0.02 * rng.standard_normal((N, HV, D, D))).astype(np.float32)
+    eps = 1e-3                                                                  # the Qwen3-next page's value
+    z, wn = I.outgate_inputs(n_pre + 2 * N, HV, D, io, 88)                     # prefill rows, then decode rows
+    zd = to_dev(z).view(n_pre + 2 * N, HV, D)
+    wnd = to_dev(wn)
 
     # ---- GPU: convolution, gates, prefill, then two decode steps from raw projections
     q, k, v, cs = _gpu_conv(x, w, st0, bounds, 1, n_pre, HK, HV, D, act)
@@ -156,14 +162,19 @@ def test_conv_prefill_decode_end_to_end():
     Ad, dd = to_dev(A_log), to_dev(dt_bias)
     g, beta = G.gdn_gates(ad[:n_pre].view(1, n_pre, HV), bd[:n_pre].view(1, n_pre, HV), Ad, dd)
     cud = to_dev(bounds.astype(np.int32))
-    o_pre, hT = G.gdn_chunk_prefill(q, k, v, g, beta, initial_state=to_dev(h0), cu_seqlens=cud)
+    if outgate:
+        o_pre, hT = G.gdn_chunk_prefill_outgate(q, k, v, g, beta, zd[:n_pre].view(1, n_pre, HV, D), wnd, eps,
+                                                initial_state=to_dev(h0), cu_seqlens=cud)
+    else:
+        o_pre, hT = G.gdn_chunk_prefill(q, k, v, g, beta, initial_state=to_dev(h0), cu_seqlens=cud)
     wd = to_dev(w)
     cs_next = torch.empty_like(cs)
     o_dec = []
     for s in range(2):
         rows = slice(n_pre + s * N, n_pre + (s + 1) * N)
+        og = (zd[rows].contiguous(), wnd, eps) if outgate else None
         o_s, _ = G.gdn_decode_step_fused(to_dev(xdec).view(2 * N, -1)[s * N:(s + 1) * N], wd, cs, ad[rows], bd[rows],
-                                         Ad, dd, hT, HK=HK, conv_act=act, conv_state_out=cs_next)
+                                         Ad, dd, hT, HK=HK, conv_act=act, conv_state_out=cs_next, outgate=og)
         o_dec.append(to_np(o_s))
         cs, cs_next = cs_next, cs
     assert G.gdn_decode_status() == 0
@@ -185,6 +196,8 @@ def test_conv_prefill_decode_end_to_end():
     g_ref, beta_ref = oracle.gates(a[order].astype(np.float64), b[order].astype(np.float64),
                                    A_log.astype(np.float64), dt_bias.astype(np.float64))
     o_ref, hT_ref = oracle.recurrence(qr, kr, vr, g_ref, beta_ref, h0=h0, cu_seqlens=full_bounds)
+    if outgate:
+        o_ref = oracle.out_gate(o_ref, z.f64().reshape(n_pre + 2 * N, HV, D)[order], wn.astype(np.float64), eps=eps)
     tol = TOL[io]
     assert_close(to_np(o_pre).reshape(n_pre, HV, D), o_ref[pre_rows], tol, "prefill o", out_bf16=True)
     for s in range(2):
@@ -192,3 +205,13 @@ def test_conv_prefill_decode_end_to_end():
         assert_close(o_dec[s], o_ref[dec_rows], tol, f"decode step {s} o", out_bf16=True)
     assert_close(to_np(hT), hT_ref, tol, "final state")
     np.testing.assert_array_equal(to_np(cs).transpose(0, 2, 1), st_ref, err_msg="conv state after decoding")
+
+
+def test_conv_prefill_decode_end_to_end():
+    _end_to_end(outgate=False)
+
+
+def test_conv_prefill_decode_end_to_end_output_epilogue():
+    """The same sequences with the output epilogue on the prefill and on both decode steps:
+    the two calls apply one epilogue, so the decoded tokens continue the prefilled ones."""
+    _end_to_end(outgate=True)
