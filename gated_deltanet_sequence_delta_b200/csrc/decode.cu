@@ -226,13 +226,9 @@ decode_staged_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
         tc::fence_mbar_init();
     }
     __syncthreads();
-    // Launched with programmatic stream serialisation: this grid may start while the kernel
-    // before it in the stream is still running.  Nothing in global memory is touched before
-    // that kernel has completed and its writes are visible; then the next grid may launch, its
-    // CTAs taking each SM as this grid's CTA there exits (every CTA of this grid is resident
-    // by then, so a waiting CTA of the next grid never holds an SM this grid still needs).
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // launched with programmatic stream serialisation: the next step's CTAs take each SM as
+    // this grid's CTA there exits (tc::grid_dependency_sync)
+    tc::grid_dependency_sync();
 
     if (warp == kSWarps) {
         // ---------------- producer ----------------------------------------------------

@@ -135,6 +135,18 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     }
 }
 
+// ---- programmatic dependent launch ----------------------------------------------------
+// For kernels launched with programmatic stream serialisation, which may start while the
+// kernel before them in the stream is still running: wait until that kernel has completed
+// and its writes are visible (before any global-memory access), then let the next such
+// kernel launch.  The next grid launches only once every CTA of this one has signalled or
+// exited, so all of this grid's CTAs are resident by then and a waiting CTA of the next
+// grid never holds an SM this grid still needs.
+__device__ __forceinline__ void grid_dependency_sync() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- proxies and TMEM ordering fences ------------------------------------------------
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
