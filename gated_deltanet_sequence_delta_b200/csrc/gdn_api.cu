@@ -100,7 +100,6 @@ size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seqs, int32
     if (n_tokens < 0 || n_tokens > INT32_MAX || n_seqs < 0 || HK <= 0 || HV <= 0 || HV % HK != 0) return 0;
     if (!head_dim_ok(Dk) || !head_dim_ok(Dv) || !dtype_ok(io_dtype)) return 0;
     if (!(BT == 16 || BT == 32 || BT == 64)) return 0;
-    if (io_dtype == GDN_BF16 && BT != 64) return 0;
     if (io_dtype == GDN_BF16 && gdn::prefill_tc_supported(Dk, Dv, HK, HV, BT))
         return gdn::prefill_tc_workspace_bytes(n_tokens, n_seqs, HK, HV);
     return gdn::kStatusBytes;

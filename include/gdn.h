@@ -127,10 +127,10 @@ GDN_API size_t gdn_chunk_prefill_workspace_bytes(int64_t n_tokens, int32_t n_seq
  *   workspace     device scratch of >= gdn_chunk_prefill_workspace_bytes(...) bytes,
  *                 owned by the caller, contents need not be initialised; it must
  *                 not be shared by calls that may run concurrently.
- *   BT            chunk length: 64 (GDN_BF16) or 16, 32, 64 (GDN_F32).  BT only
- *                 changes rounding, never the result's definition.
- *                 GDN_BF16 with Dk = Dv = 128 and HV / HK in {1, 2, 4} runs on the tensor
- *                 cores (tcgen05); other GDN_BF16 shapes and GDN_F32 run on CUDA cores.
+ *   BT            chunk length: 16, 32 or 64.  BT only changes rounding, never the
+ *                 result's definition.
+ *                 GDN_BF16 with Dk = Dv = 128, HV / HK in {1, 2, 4} and BT = 64 runs on
+ *                 the tensor cores (tcgen05); every other configuration runs on CUDA cores.
  *   scale         multiplies o (1.0 = the plain rule).
  *   qk_l2norm     nonzero: q and k rows are replaced by x / sqrt(sum x^2 + 1e-6)
  *                 before use (per token and q/k head).

@@ -57,7 +57,7 @@ def test_prefill_validation(L):
     assert _prefill(L, B=2, N=1) == 2                     # dense needs N == B
     assert _prefill(L, cu=A + 500 * MB, B=2, N=2) == 2    # packed needs B == 1
     assert _prefill(L, Dk=96) == 4                        # unsupported head dim
-    assert _prefill(L, BT=32) == 4                        # bf16 path needs BT = 64
+    assert _prefill(L, BT=48) == 4                        # chunk length not 16, 32 or 64
     assert _prefill(L, io=1, BT=128) == 4
     assert _prefill(L, ws=None) == 6
     assert _prefill(L, ws_bytes=16) == 6
@@ -301,7 +301,7 @@ def test_static_scratch_entry_point_reports_sizes_like_the_workspace_one(L):
                  a["N"], a["HK"], a["HV"], a["Dk"], a["Dv"], a["BT"], 1.0, 1, A + 256 * MB, A + 384 * MB, None)
 
     cases = [dict(HK=2, HV=3), dict(HK=0), dict(B=2, N=1), dict(cu=A + 500 * MB, B=2, N=2), dict(Dk=96),
-             dict(BT=32), dict(T=-1), dict(io=5), dict(cu=A + 500 * MB, T=1 << 31)]
+             dict(BT=48), dict(T=-1), dict(io=5), dict(cu=A + 500 * MB, T=1 << 31)]
     for kw in cases:
         want = _prefill(L, **{k: v for k, v in kw.items() if k != "io"}, **({"io": kw["io"]} if "io" in kw else {}))
         assert want != 0, kw

@@ -83,6 +83,25 @@ def test_bt_independence_fp32():
         assert_close(to_np(hT), to_np(outs[0][1]), 1e-5, "state across BT")
 
 
+def test_bt_independence_bf16():
+    """bf16 with 128-dim heads: BT = 64 on the tensor cores (fp16 intermediates), BT = 32
+    and 16 on CUDA cores (fp32 throughout).  Each agrees with the oracle within the bf16
+    bound; the two CUDA-core chunk lengths give the same fp32 final state to fp32 accuracy
+    (the chunk length changes only where sums are rounded).  Their bf16 outputs are not
+    compared with each other: two roundings of nearly equal values may land one bf16 step
+    apart, more than the half step the bound allows against the exact result."""
+    inp = I.make_prefill(2, 333, 2, 4, 128, 128, io_dtype=I.BF16, seed=13, h0_std=0.05)
+    o_ref, h_ref = oracle_prefill(inp)
+    tol = TOL[I.BF16]
+    outs = {}
+    for bt in (64, 32, 16):
+        o, hT, _, _ = gpu_prefill(inp, BT=bt)
+        assert_close(to_np(o), o_ref, tol, f"bf16, BT {bt}: o", out_bf16=True)
+        assert_close(to_np(hT), h_ref, tol, f"bf16, BT {bt}: final state")
+        outs[bt] = (to_np(o), to_np(hT))
+    assert_close(outs[16][1], outs[32][1], TOL[I.F32], "bf16 state, BT 16 against BT 32")
+
+
 @pytest.mark.parametrize("io", [I.F32, I.BF16])
 def test_varlen_equals_separate_calls(io):
     import gated_deltanet_sequence_delta_b200 as G
