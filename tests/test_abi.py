@@ -125,6 +125,15 @@ def test_prefill_workspace_query(L):
     assert L.gdn_chunk_prefill_workspace_bytes(2 ** 31, 1, 16, 32, 128, 128, 64, 1) == 0
     assert L.gdn_chunk_prefill_workspace_bytes(2 ** 26, 1, 32, 32, 128, 128, 64, 1) == 0
     assert L.gdn_chunk_prefill_workspace_bytes(2 ** 20, 1, 32, 32, 128, 128, 64, 1) > 0
+    # chunk lengths: 16, 32 and 64 in both dtypes; bf16 at 16 or 32 takes the CUDA-core path,
+    # whose workspace is the status word alone, far less than the tensor-core path's tiles
+    tc = L.gdn_chunk_prefill_workspace_bytes(4096, 1, 2, 4, 128, 128, 64, 1)
+    for bt in (16, 32):
+        cc = L.gdn_chunk_prefill_workspace_bytes(4096, 1, 2, 4, 128, 128, bt, 1)
+        assert 0 < cc < tc, (bt, cc, tc)
+        assert L.gdn_chunk_prefill_workspace_bytes(4096, 1, 2, 4, 128, 128, bt, 0) > 0
+    for bt in (8, 48, 128):
+        assert L.gdn_chunk_prefill_workspace_bytes(4096, 1, 2, 4, 128, 128, bt, 1) == 0
 
 
 def test_gates_validation(L):
